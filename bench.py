@@ -1,0 +1,503 @@
+#!/usr/bin/env python
+"""Benchmark of the paged-KV attention hot path on B200.
+
+Default (N=1): one layer of Qwen3-0.6B-shaped decode -- batch 32, context
+lengths uniform in [128, 4096], 16 query / 8 KV heads, head_dim 128, block
+size 256, shuffled pool sized 1.25x the need.  One step = store each
+sequence's new K/V row into the pool + paged decode attention over the batch.
+
+Metric: decode-step KV GB/s (algorithmic bytes of the step / step time), with
+tokens/s (sequences decoded per second for this layer) beside it.  Inputs are
+resident in HBM when timing starts; L2 is flushed (a 512 MiB write) before
+every timed step and each step is bracketed by CUDA events on the launching
+stream.  With --gpus N (torchrun, one rank per GPU) every rank runs its own
+replica of the workload (no collective on the data path: "scaling": "weak")
+and the time is the max over ranks.
+
+Also measured in the same run and reported under "workloads": 7B-GQA decode
+(batch 256, 28/4 heads, block 256 and block 16), the prefix-cached prefill
+(TFLOP/s), a large store_kvcache (GB/s) and the continuous-batching trace
+replay (tokens/s).  ``--impl reference`` times the CPU oracle on a bounded
+sample of the same workload instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+HBM_FALLBACK_GBS = 6650.0
+BF16_FALLBACK_TFLOPS = 1590.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": HBM_FALLBACK_GBS, "bf16_tflops": BF16_FALLBACK_TFLOPS,
+            "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples nvidia-smi clocks / throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------- timing
+class Timer:
+    """Per-step CUDA-event timing on the current stream, L2 flushed before each step."""
+
+    def __init__(self, torch, flush_bytes=512 << 20):
+        self.torch = torch
+        self.flush_buf = torch.empty(flush_bytes, dtype=torch.uint8, device="cuda")
+
+    def flush(self):
+        self.flush_buf.fill_(1)
+
+    def time_steps(self, fn, steps, marks=1):
+        """Runs `fn(ev)` `steps` times; fn records its own events in `ev` (list of marks+1 events).
+        Returns per-step lists of segment durations in ms."""
+        torch = self.torch
+        segs = []
+        for _ in range(steps):
+            self.flush()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(marks + 1)]
+            fn(ev)
+            segs.append(ev)
+        torch.cuda.synchronize()
+        return [[e[i].elapsed_time(e[i + 1]) for i in range(marks)] for e in segs]
+
+
+def dist_setup():
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return torch, dist, world, rank, local
+
+
+def max_over_ranks(torch, dist, world, x: float) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(torch, dist, world):
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+# ------------------------------------------------------------ workloads (ours)
+def bench_decode(torch, w, steps, warmup, timer, dist=None, world=1, partition=0):
+    """Times `steps` decode steps; returns dict of mean ms per segment."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        w.step(partition_size=partition)
+    barrier(torch, dist, world)
+
+    def one(ev):
+        from paged_kv_attention_35_b200 import ops
+        ev[0].record(stream)
+        ops.store_kvcache(w.d_new_k, w.d_new_v, w.kc, w.vc, w.d_slots)
+        ev[1].record(stream)
+        ops.decode(w.d_q, w.kc, w.vc, w.d_bt, w.d_cl, w.max_context_len, out=w.d_out,
+                   workspace=w.d_ws, partition_size=partition)
+        ev[2].record(stream)
+
+    segs = np.asarray(timer.time_steps(one, steps, marks=2))
+    barrier(torch, dist, world)
+    return {"store_ms": float(segs[:, 0].mean()), "decode_ms": float(segs[:, 1].mean()),
+            "step_ms": float(segs.sum(axis=1).mean()), "step_ms_total": float(segs.sum())}
+
+
+def bench_decode_e2e(torch, w, steps, warmup, timer):
+    """Same step through host buffers: H2D of the step's inputs, kernels, D2H of the output."""
+    from paged_kv_attention_35_b200 import ops
+    stream = torch.cuda.current_stream()
+    h = {
+        "q": w.q.pin_memory(), "k": w.new_k.pin_memory(), "v": w.new_v.pin_memory(),
+        "slots": torch.from_numpy(w.decode_slots).pin_memory(),
+        "bt": torch.from_numpy(w.block_tables).pin_memory(),
+        "cl": torch.tensor(w.lens, dtype=torch.int32).pin_memory(),
+    }
+    out_h = torch.empty(w.d_out.shape, dtype=torch.bfloat16).pin_memory()
+    d = {"q": w.d_q, "k": w.d_new_k, "v": w.d_new_v, "slots": w.d_slots, "bt": w.d_bt, "cl": w.d_cl}
+    h2d = sum(t.numel() * t.element_size() for t in h.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    def one(ev):
+        ev[0].record(stream)
+        for k in h:
+            d[k].copy_(h[k], non_blocking=True)
+        ops.store_kvcache(d["k"], d["v"], w.kc, w.vc, d["slots"])
+        ops.decode(d["q"], w.kc, w.vc, d["bt"], d["cl"], w.max_context_len, out=w.d_out,
+                   workspace=w.d_ws)
+        out_h.copy_(w.d_out, non_blocking=True)
+        ev[1].record(stream)
+
+    for _ in range(warmup):
+        timer.time_steps(one, 1)
+    segs = np.asarray(timer.time_steps(one, steps))
+    return float(segs.mean()), h2d, d2h
+
+
+def bench_prefill(torch, steps, warmup, timer):
+    from paged_kv_attention_35_b200.workloads import PrefixPrefillWorkload
+    from paged_kv_attention_35_b200 import synth
+    w = PrefixPrefillWorkload(seed=synth.SEED_BASE + 4).upload("cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        w.step()
+
+    def one(ev):
+        ev[0].record(stream)
+        w.store()
+        ev[1].record(stream)
+        w.attend()
+        ev[2].record(stream)
+
+    segs = np.asarray(timer.time_steps(one, steps, marks=2))
+    store_ms, attn_ms = float(segs[:, 0].mean()), float(segs[:, 1].mean())
+    return w, store_ms, attn_ms
+
+
+def bench_store_large(torch, steps, warmup, timer):
+    """N = 65536 new tokens, Hkv 8, D 128, block 256, slots a seeded permutation of the pool."""
+    from paged_kv_attention_35_b200 import ops, synth
+    n, hkv, d, bs = 65536, 8, 128, 256
+    nb = n // bs
+    key = synth.bf16_normal((n, hkv, d), 7).cuda()
+    val = synth.bf16_normal((n, hkv, d), 8).cuda()
+    kc = torch.empty((nb, bs, hkv, d), dtype=torch.bfloat16, device="cuda")
+    vc = torch.empty_like(kc)
+    slots = torch.from_numpy(synth.permutation(nb * bs, 9).astype(np.int32)).cuda()
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        ops.store_kvcache(key, val, kc, vc, slots)
+
+    def one(ev):
+        ev[0].record(stream)
+        ops.store_kvcache(key, val, kc, vc, slots)
+        ev[1].record(stream)
+
+    ms = float(np.asarray(timer.time_steps(one, steps)).mean())
+    nbytes = 2 * 2 * n * hkv * d * 2
+    return nbytes, ms
+
+
+def ours(args):
+    torch, dist, world, rank, local = dist_setup()
+    from paged_kv_attention_35_b200 import ops  # noqa: F401  (fails loudly without the library)
+    from paged_kv_attention_35_b200 import synth
+    from paged_kv_attention_35_b200.workloads import DecodeWorkload
+    pk = peaks()
+    timer = Timer(torch)
+    spec = synth.WORKLOADS[args.workload]
+    w = DecodeWorkload.from_spec(spec).upload("cuda")
+    launches_per_step = 2 + (1 if ops.decode_workspace_size(
+        w.B, w.hq, w.hkv, w.d, w.max_context_len, args.partition) > 0 else 0)
+
+    with ClockSampler(local) as clk:
+        r = bench_decode(torch, w, args.steps, args.warmup, timer, dist, world, args.partition)
+    # max over ranks of the timed region (sum of the K steps' device time)
+    total_ms = max_over_ranks(torch, dist, world, r["step_ms_total"])
+    step_ms = total_ms / args.steps
+    step_bytes = w.step_bytes()
+    value = world * step_bytes * args.steps / (total_ms * 1e-3) / 1e9
+    tokens_s = world * w.B * args.steps / (total_ms * 1e-3)
+    decode_gbs = w.kv_bytes() / (r["decode_ms"] * 1e-3) / 1e9
+
+    e2e_ms, h2d, d2h = bench_decode_e2e(torch, w, args.steps, args.warmup, timer)
+    e2e_ms = max_over_ranks(torch, dist, world, e2e_ms)
+
+    extra = {}
+    if not args.quick and rank == 0:
+        extra = secondary(torch, args, timer, pk)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline_decode(w, budget_s=args.cpu_budget)
+
+    if rank == 0:
+        traffic = load_traffic("decode_kernel", args.workload)
+        line = {
+            "metric": "paged decode attention KV GB/s (decode step: store_kvcache + decode)",
+            "value": round(value, 1),
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(step_ms, 4),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 K/V/q, seeded context lengths and shuffled pool)",
+            "config": {"workload": spec.name, "num_seqs": w.B, "context_lens": "U[128,4096]",
+                       "sum_context": int(sum(w.lens)), "num_q_heads": w.hq, "num_kv_heads": w.hkv,
+                       "head_dim": w.d, "block_size": w.bs, "num_blocks": w.nb,
+                       "partition": args.partition or "auto", "l2": "flushed (512 MiB write) before every step",
+                       "parallelism": f"replicas x{world}"},
+            "tokens_per_s": round(tokens_s, 1),
+            "breakdown_ms": {"store_kvcache": round(r["store_ms"], 4), "decode": round(r["decode_ms"], 4)},
+            "roofline": {"bound": "hbm", "kernel": "pa_decode (split-K decode + merge)",
+                         "achieved": round(decode_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(decode_gbs / pk["hbm_gbs"], 4),
+                         "peak_source": pk["source"], "traffic": traffic},
+            "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                    "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+            "workloads": extra,
+            "pages_context": {"qwen7b_tokens_per_s": {"bs1": 32, "bs8": 215, "bs16": 398},
+                              "note": "end-to-end model throughput quoted by the pages, hardware not stated"},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def secondary(torch, args, timer, pk):
+    """The other workloads, each at its own roofline (rank 0, N=1 or any N)."""
+    from paged_kv_attention_35_b200 import synth
+    from paged_kv_attention_35_b200.workloads import DecodeWorkload
+    out = {}
+    steps = max(3, min(args.steps, 10))
+    for bs in (256, 16):
+        w = DecodeWorkload.from_spec(synth.WORKLOADS["gqa7b_decode"], block_size=bs).upload("cuda")
+        r = bench_decode(torch, w, steps, 3, timer)
+        gbs = w.kv_bytes() / (r["decode_ms"] * 1e-3) / 1e9
+        out[f"gqa7b_decode_bs{bs}"] = {
+            "step_ms": round(r["step_ms"], 4), "decode_ms": round(r["decode_ms"], 4),
+            "store_ms": round(r["store_ms"], 4), "kv_bytes": w.kv_bytes(),
+            "decode_GBs": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4),
+            "tokens_per_s": round(w.B / (r["step_ms"] * 1e-3), 1)}
+        del w
+        torch.cuda.empty_cache()
+    w, store_ms, attn_ms = bench_prefill(torch, steps, 3, timer)
+    tf = w.flops() / (attn_ms * 1e-3) / 1e12
+    out["prefix_prefill"] = {
+        "attn_ms": round(attn_ms, 4), "store_ms": round(store_ms, 4), "flops": w.flops(),
+        "total_q": int(w.md.total_q), "TFLOPs": round(tf, 1),
+        "frac_bf16_peak": round(tf / pk["bf16_tflops"], 4),
+        "frac_bf16_sustained": round(tf / pk["bf16_tflops_sustained"], 4),
+        "store_GBs": round(w.store_bytes() / (store_ms * 1e-3) / 1e9, 1)}
+    del w
+    torch.cuda.empty_cache()
+    nbytes, ms = bench_store_large(torch, steps, 3, timer)
+    out["store_kvcache_65536"] = {"ms": round(ms, 4), "bytes": nbytes,
+                                  "GBs": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                                  "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+    torch.cuda.empty_cache()
+    if not args.no_replay:
+        try:
+            from paged_kv_attention_35_b200.replay import run_replay_bench
+            out["trace_replay"] = run_replay_bench(torch, max_steps=args.replay_steps)
+        except ImportError:
+            pass
+    return out
+
+
+def load_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch recorded from an ncu capture of this kernel and workload, if any."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    return d.get(f"{kernel}:{workload}")
+
+
+# ------------------------------------------------------------ CPU oracle arm
+def decode_sample_inputs(w, rows):
+    """Oracle inputs (float64) for sequences `rows` of a decode workload: q, and a
+    compact pool holding only their blocks (renumbered), built from the logical draws."""
+    import oracle
+    import torch
+
+    def bits(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    lens = [w.lens[i] for i in rows]
+    nblk = [-(-L // w.bs) for L in lens]
+    bt = np.full((len(rows), max(nblk)), -1, np.int32)
+    kp = np.zeros((sum(nblk), w.bs, w.hkv, w.d), np.uint16)
+    vp = np.zeros_like(kp)
+    k = 0
+    for j, i in enumerate(rows):
+        bt[j, :nblk[j]] = np.arange(k, k + nblk[j])
+        flat_k = kp[k:k + nblk[j]].reshape(-1, w.hkv, w.d)
+        flat_v = vp[k:k + nblk[j]].reshape(-1, w.hkv, w.d)
+        flat_k[:lens[j]] = bits(w.k[i])
+        flat_v[:lens[j]] = bits(w.v[i])
+        k += nblk[j]
+    q = oracle.bf16_bits_to_f64(bits(w.q))[rows]
+    return q, oracle.bf16_bits_to_f64(kp), oracle.bf16_bits_to_f64(vp), bt, np.asarray(lens)
+
+
+def cpu_baseline_decode(w, budget_s=15.0):
+    """Time the oracle (as it stands) on a bounded sample of the decode workload."""
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    t_start = time.perf_counter()
+    done_bytes = 0
+    n = 0
+    order = list(range(w.B))
+    t_or = 0.0
+    while time.perf_counter() - t_start < budget_s and n < len(order):
+        i = order[n]
+        q, kp, vp, bt, lens = decode_sample_inputs(w, [i])
+        t0 = time.perf_counter()
+        oracle.ref_decode(q, kp, vp, bt, lens)
+        t_or += time.perf_counter() - t0
+        done_bytes += w.lens[i] * w.hkv * w.d * 2 * 2
+        n += 1
+    gbs = done_bytes / t_or / 1e9 if t_or > 0 else None
+    return {"value": gbs, "unit": "GB/s", "cores": _blas_threads(cores), "kind": "oracle",
+            "sample": f"{n} of {w.B} sequences (all {w.hq} heads), oracle time {t_or:.2f} s",
+            "seconds": round(t_or, 2)}
+
+
+def _blas_threads(default):
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        if info:
+            return max(int(i.get("num_threads", 1)) for i in info)
+    except Exception:
+        pass
+    return default
+
+
+def reference(args):
+    """The oracle as the reference arm: same metric/config, bounded sample per step."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from paged_kv_attention_35_b200 import synth
+    from paged_kv_attention_35_b200.workloads import DecodeWorkload
+    spec = synth.WORKLOADS[args.workload]
+    w = DecodeWorkload.from_spec(spec)
+    budget = max(1.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline_decode(w, budget_s=budget)
+    vals = []
+    last = None
+    for _ in range(args.steps):
+        last = cpu_baseline_decode(w, budget_s=budget)
+        vals.append(last["value"])
+    v = float(np.mean(vals))
+    line = {
+        "impl": "reference", "metric": "paged decode attention KV GB/s (decode step: store_kvcache + decode)",
+        "value": round(v, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (same seeded workload)",
+        "config": {"workload": spec.name, "num_seqs": w.B, "num_q_heads": w.hq,
+                   "num_kv_heads": w.hkv, "head_dim": w.d, "block_size": w.bs},
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "kind": "oracle",
+                         "cores": last["cores"], "sample": last["sample"]},
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen3_0p6b_decode")
+    ap.add_argument("--partition", type=int, default=0)
+    ap.add_argument("--quick", action="store_true", help="primary workload only")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-replay", action="store_true")
+    ap.add_argument("--replay-steps", type=int, default=0)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        reference(args)
+    else:
+        ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,197 @@
+/*
+ * pagedattn.h -- C ABI of libpagedattn.so, the paged-KV attention hot path of a
+ * nano-vLLM-style serving engine, for NVIDIA B200 (sm_100a).
+ *
+ * What the pages fix.  "Deep into the Nano-vLLM inference engine" (lnwmold.com
+ * news item), section "Control plane vs. data plane": the block manager is a
+ * CPU-side control plane that only tracks metadata, while the KV cache itself
+ * lives on the GPU (the data plane); freed blocks are marked free and their GPU
+ * memory is not cleared.  "Nano-vLLM engine architecture" (intelliparadigm.com)
+ * section 3.2: GPU memory is cut into fixed-size blocks (default 256 tokens).
+ * The same lnwmold.com item, section "Preparation before computation": a
+ * prefill batches sequences by cumulative sequence lengths; a decode batches
+ * one new token per sequence.  This library is that data plane.
+ *
+ * Layouts (readings; the pages defer the physical layout, section "What's
+ * Next" of the lnwmold.com item):
+ *   K pool, V pool   [num_blocks, block_size, num_kv_heads, head_dim]  bf16
+ *                    slot s = flat token row s of [num_blocks*block_size, Hkv, D]
+ *   key / value      [N, num_kv_heads, head_dim] bf16, rows key_token_stride apart
+ *   q (decode)       [num_seqs, num_q_heads, head_dim] bf16, rows q_token_stride apart
+ *   q (prefill)      [total_q, num_q_heads, head_dim] bf16, rows q_token_stride apart
+ *   out              [rows, num_q_heads, head_dim] bf16, contiguous
+ *   block_tables     [num_seqs, max_blocks_per_seq] int32 (unused entries: any value)
+ *   GQA              query head h reads KV head h / (num_q_heads / num_kv_heads)
+ *
+ * Ownership.  The caller allocates and owns every buffer (including the decode
+ * workspace).  The library never allocates, frees or synchronises; all work is
+ * enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream) and
+ * the buffers must stay alive until it has run.  Pointers are device pointers
+ * to 16-byte aligned memory; head_dim is innermost and contiguous.
+ *
+ * Errors.  Host-side validation runs before any launch and returns a status;
+ * pa_last_error_message() gives the reason (thread-local).  A launch failure
+ * returns PA_ERR_CUDA.  Device-side metadata checks: with a non-NULL err_flag
+ * (device int32), kernels OR a PA_FLAG_* bit into it when metadata is out of
+ * range and skip or neutralise the offending access; they never trap.  With a
+ * NULL err_flag the same guards still keep every access inside the buffers
+ * (out-of-range block ids read zeros), but nothing is reported.  Every wait in
+ * the kernels is bounded: a wait that gives up (about two seconds) sets
+ * PA_FLAG_TIMEOUT (in err_flag, and in a device-global word read by
+ * pa_watchdog_read) and the kernel returns.
+ *
+ * Threading: the entry points are re-entrant; a per-(pointer, shape) cache of
+ * TMA tensor maps is guarded by a mutex.
+ */
+#ifndef PAGEDATTN_H
+#define PAGEDATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,   /* a size, pointer or alignment is invalid             */
+  PA_ERR_UNSUPPORTED = 2,   /* valid, but outside what the kernels implement        */
+  PA_ERR_WORKSPACE = 3,     /* decode workspace missing or smaller than required    */
+  PA_ERR_CUDA = 4           /* a CUDA runtime/driver call or a launch failed        */
+} pa_status;
+
+typedef enum { PA_BF16 = 0 } pa_dtype;
+
+/* bits OR-ed into *err_flag (checked mode) */
+#define PA_FLAG_SLOT_OOB   1  /* slot_mapping entry >= num_blocks*block_size          */
+#define PA_FLAG_BLOCK_OOB  2  /* block table entry outside [0, num_blocks)            */
+#define PA_FLAG_LEN_OOB    4  /* context/sequence length outside its declared bounds  */
+#define PA_FLAG_TIMEOUT    8  /* a bounded wait gave up                                */
+
+typedef void* pa_stream_t;
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+/* Human-readable name of a status. Never NULL. */
+PA_API const char* pa_status_string(pa_status s);
+
+/* Detail of the last non-OK status returned on this thread ("" if none). */
+PA_API const char* pa_last_error_message(void);
+
+/* Library version string, e.g. "pagedattn 0.1 sm_100a". */
+PA_API const char* pa_version(void);
+
+/*
+ * pa_store_kvcache -- scatter each step's new K/V rows into the block pool.
+ *
+ * For i in [0, num_tokens): if slot_mapping[i] >= 0, copies key row i to flat
+ * token row slot_mapping[i] of k_cache and value row i to the same row of
+ * v_cache (num_kv_heads*head_dim bf16 each, bit-exact).  A negative slot means
+ * padding: nothing is written.  Source: the Block Manager hands every token a
+ * place in a fixed-size block ("From Sequences to Blocks", lnwmold.com item);
+ * the new token's cache is written before attention reads it ("Handling
+ * resource exhaustion": room for the next token's cache).
+ *   key, value           device, [num_tokens, Hkv, D], rows *_token_stride
+ *                        elements apart (>= Hkv*D, multiple of 8)
+ *   k_cache, v_cache     device, [num_slots, Hkv, D] (num_slots = NB*block_size)
+ *   slot_mapping         device int32 [num_tokens]
+ *   Hkv*D must be a multiple of 8 (16-byte rows).  num_tokens == 0 is a no-op.
+ * Rows that name the same slot race (the caller's control plane never does
+ * that).  Slots >= num_slots are skipped (PA_FLAG_SLOT_OOB in checked mode).
+ */
+PA_API pa_status pa_store_kvcache(const void* key, const void* value,
+                           int64_t key_token_stride, int64_t value_token_stride,
+                           void* k_cache, void* v_cache,
+                           const int32_t* slot_mapping, int32_t num_tokens,
+                           int32_t num_kv_heads, int32_t head_dim, int64_t num_slots,
+                           pa_dtype dtype, int32_t* err_flag, pa_stream_t stream);
+
+/*
+ * pa_decode_workspace_size -- bytes of workspace pa_decode needs for these
+ * sizes (0 when no sequence can be split).  partition_size 0 = automatic
+ * (same rule pa_decode applies), else the explicit value passed to pa_decode.
+ */
+PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                int32_t head_dim, int32_t max_context_len,
+                                int32_t partition_size);
+
+/*
+ * pa_decode -- paged decode attention with GQA (one query token per sequence).
+ *
+ * For sequence i and query head h (g = h / (Hq/Hkv)):
+ *   out[i,h,:] = softmax_t(scale * q[i,h,:] . K_i[t,g,:]) @ V_i[t,g,:],
+ *   t = 0 .. context_lens[i]-1,
+ * where row t of K_i / V_i is pool row block_tables[i][t / block_size] *
+ * block_size + t % block_size.  context_lens counts the new token, whose K/V
+ * must already be stored.  bf16 inputs, fp32 accumulation, bf16 output.
+ * Source: decode batches one new token per sequence ("Preparation before
+ * computation", "Prefill and Decode", lnwmold.com item) against the paged
+ * pool (intelliparadigm.com section 3.2); the attention formula itself is not
+ * written on the pages (deferred to their part 2) and is the standard
+ * scaled-dot-product softmax attention.
+ *
+ * Long contexts are split into partitions of partition_size tokens (0 =
+ * automatic; else a multiple of 64) that run in parallel; their partial
+ * results go to `workspace` (>= pa_decode_workspace_size bytes, 256-byte
+ * aligned, caller-owned, contents need no initialisation) and a second kernel
+ * merges them.  max_context_len must bound every context_lens entry (it sizes
+ * the grid).  Supported: head_dim 64 or 128, block_size a power of two in
+ * [16, 1024], 1 <= Hq/Hkv.  context_lens[i] == 0 gives a zero output row
+ * (PA_FLAG_LEN_OOB in checked mode).
+ */
+PA_API pa_status pa_decode(void* out, const void* q, int64_t q_token_stride,
+                    const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq,
+                    const int32_t* context_lens, int32_t num_seqs, int32_t max_context_len,
+                    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                    int32_t block_size, int32_t num_blocks, float scale,
+                    int32_t partition_size, void* workspace, size_t workspace_bytes,
+                    pa_dtype dtype, int32_t* err_flag, pa_stream_t stream);
+
+/*
+ * pa_prefill_varlen -- causal prefill over prompts packed by cumulative
+ * sequence lengths, reading K/V from the paged pool (prefix-cached blocks
+ * included).
+ *
+ * Sequence i computes q_len = cu_seqlens_q[i+1]-cu_seqlens_q[i] new queries
+ * and has k_len = cu_seqlens_k[i+1]-cu_seqlens_k[i] keys (k_len >= q_len);
+ * the first k_len-q_len keys are a cached prefix (blocks shared through the
+ * hash prefix cache, "Prefix Caching via hashing", lnwmold.com item).  Query
+ * j sits at absolute position k_len-q_len+j and attends keys 0 .. that
+ * position (bottom-right causal alignment):
+ *   out[r,h,:] = softmax_t(scale * q[r,h,:] . K_i[t,g,:]) @ V_i[t,g,:].
+ * All K/V rows -- the new tokens' included -- are read from the pool, so the
+ * step's pa_store_kvcache must be enqueued first on the same stream.
+ *   q          device [total_q, Hq, D], rows q_token_stride elements apart
+ *   out        device [total_q, Hq, D] contiguous
+ *   cu_seqlens device int32 [num_seqs+1], starting at 0
+ *   max_seqlen_q / max_seqlen_k bound every q_len / k_len (they size the grid)
+ * Supported: head_dim 128 (tensor-core path) or 64, block_size a power of two
+ * in [16, 1024].
+ */
+PA_API pa_status pa_prefill_varlen(void* out, const void* q, int64_t q_token_stride,
+                            const void* k_cache, const void* v_cache,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                            int32_t max_seqlen_q, int32_t max_seqlen_k, int32_t total_q,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq,
+                            int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                            int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                            float scale, pa_dtype dtype, int32_t* err_flag, pa_stream_t stream);
+
+/*
+ * pa_watchdog_read -- copy (and clear) the device-global word where kernels
+ * launched without err_flag record PA_FLAG_TIMEOUT.  Synchronous on the
+ * current device.  Returns PA_ERR_CUDA if the copy fails.
+ */
+PA_API pa_status pa_watchdog_read(uint32_t* value);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_H */

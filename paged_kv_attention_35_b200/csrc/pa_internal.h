@@ -1,0 +1,76 @@
+// pa_internal.h -- host-side pieces shared by the library's translation units:
+// the thread-local error message, TMA tensor-map encoding for the KV pools, and
+// the kernel launchers behind the C ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/pagedattn.h"
+
+namespace pa {
+
+// Records `msg` as this thread's last error and returns `s`.
+pa_status fail(pa_status s, const std::string& msg);
+pa_status cuda_fail(cudaError_t e, const char* what);
+
+// A 3-D view [rows, heads, head_dim] of a bf16 buffer (a KV pool or packed q)
+// as a TMA tensor map with 128-byte swizzle and boxes of {64, 1, box_rows}.
+// Cached per (pointer, shape, box); thread-safe.  Fills *out on success.
+pa_status get_tensor_map(CUtensorMap* out, const void* base, int64_t rows, int heads, int head_dim,
+                         int64_t row_stride_elems, int box_rows);
+
+struct DecodeArgs {
+  void* out;
+  const void* q;
+  int64_t q_stride;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_tables;
+  int max_blocks;
+  const int32_t* context_lens;
+  int num_seqs;
+  int max_context_len;
+  int hq, hkv, d, block_size, num_blocks;
+  float scale;
+  int partition;       // tokens per partition (multiple of 64)
+  int max_splits;      // ceil(max_context_len / partition)
+  float* ws_o;         // [B, Hq, max_splits, D]
+  float* ws_ml;        // [B, Hq, max_splits, 2]
+  int32_t* err_flag;
+  cudaStream_t stream;
+};
+
+int decode_auto_partition(int num_seqs, int num_kv_heads, int max_context_len);
+pa_status launch_decode(const DecodeArgs& a);
+
+pa_status launch_store(const void* key, const void* value, int64_t key_stride,
+                       int64_t value_stride, void* k_cache, void* v_cache,
+                       const int32_t* slots, int num_tokens, int row_elems, int64_t num_slots,
+                       int32_t* err_flag, cudaStream_t stream);
+
+struct PrefillArgs {
+  void* out;
+  const void* q;
+  int64_t q_stride;
+  int total_q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int max_seqlen_q, max_seqlen_k;
+  const int32_t* block_tables;
+  int max_blocks;
+  int num_seqs;
+  int hq, hkv, d, block_size, num_blocks;
+  float scale;
+  int32_t* err_flag;
+  cudaStream_t stream;
+};
+
+pa_status launch_prefill(const PrefillArgs& a);
+
+}  // namespace pa
