@@ -154,6 +154,41 @@ PA_API pa_status pa_decode(void* out, const void* q, int64_t q_token_stride,
                     pa_dtype dtype, int32_t* err_flag, pa_stream_t stream);
 
 /*
+ * pa_decode_noalloc -- pa_decode for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this entry point; it exists for library
+ * users.  pa_decode needs a caller-allocated workspace for long contexts.
+ * Some callers cannot allocate one: an engine that reserves all GPU memory for
+ * its KV pool at start-up and must not call cudaMalloc afterwards (the call
+ * can fail once the pool owns the memory, and cudaFree synchronises the
+ * device), or a C host program that only receives ready-made device buffers
+ * from another component and has no allocator of its own.  This entry point
+ * takes the same arguments as pa_decode minus the workspace and uses a fixed
+ * scratch array owned by the library instead: a static device array of
+ * PA_DECODE_NOALLOC_SCRATCH_BYTES (16 MiB) that every GPU which loads the
+ * library holds until the process exits.  It calls no cudaMalloc, cudaFree or
+ * other allocating routine.
+ *   - Sizes whose split-K workspace (pa_decode_workspace_size) exceeds the
+ *     scratch are rejected with PA_ERR_WORKSPACE before any launch; a larger
+ *     partition_size shrinks the need.
+ *   - The first call on each device (with that device current) looks up the
+ *     scratch array's device address once (cudaGetSymbolAddress); make that
+ *     first call before any stream capture.
+ *   - Every call shares the one array, which keeps the last call's contents
+ *     (nothing in it needs to start at zero).  Calls that overlap on the GPU --
+ *     on two streams at once, or from two host threads -- race on it.
+ */
+#define PA_DECODE_NOALLOC_SCRATCH_BYTES (16u << 20)
+PA_API pa_status pa_decode_noalloc(void* out, const void* q, int64_t q_token_stride,
+                                   const void* k_cache, const void* v_cache,
+                                   const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                   const int32_t* context_lens, int32_t num_seqs,
+                                   int32_t max_context_len, int32_t num_q_heads,
+                                   int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                   int32_t num_blocks, float scale, int32_t partition_size,
+                                   pa_dtype dtype, int32_t* err_flag, pa_stream_t stream);
+
+/*
  * pa_prefill_varlen -- causal prefill over prompts packed by cumulative
  * sequence lengths, reading K/V from the paged pool (prefix-cached blocks
  * included).

@@ -42,6 +42,8 @@ SIGNATURES = {
     "pa_decode_workspace_size": ([_i32, _i32, _i32, _i32, _i32, _i32], _sz),
     "pa_decode": ([_p, _p, _i64, _p, _p, _p, _i32, _p, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
                    _f32, _i32, _p, _sz, ctypes.c_int, _p, _p], ctypes.c_int),
+    "pa_decode_noalloc": ([_p, _p, _i64, _p, _p, _p, _i32, _p, _i32, _i32, _i32, _i32, _i32, _i32,
+                           _i32, _f32, _i32, ctypes.c_int, _p, _p], ctypes.c_int),
     "pa_prefill_varlen": ([_p, _p, _i64, _p, _p, _p, _p, _i32, _i32, _i32, _p, _i32, _i32, _i32, _i32,
                            _i32, _i32, _i32, _f32, ctypes.c_int, _p, _p], ctypes.c_int),
     "pa_watchdog_read": ([ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
@@ -153,6 +155,34 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len, sca
                           int(partition_size), _ptr(workspace),
                           0 if workspace is None else workspace.numel() * workspace.element_size(),
                           PA_BF16, _ptr(err_flag), _stream()), "pa_decode")
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale=None,
+                   out=None, partition_size=0, err_flag=None):
+    """``decode`` through ``pa_decode_noalloc``: the split-K scratch is the library's
+    fixed 16 MiB device array, so no workspace is allocated or passed (for callers
+    that cannot allocate device memory).  Calls overlapping on the GPU race on it."""
+    _need_cuda(q=q, k_cache=k_cache, v_cache=v_cache, block_tables=block_tables,
+               context_lens=context_lens, out=out, err_flag=err_flag)
+    _need_bf16(q=q, k_cache=k_cache, v_cache=v_cache)
+    _need_i32(block_tables=block_tables, context_lens=context_lens)
+    nb, bs, hkv, d = k_cache.shape
+    B, hq, dq = q.shape
+    if dq != d:
+        raise ValueError("q head_dim differs from the pool's")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, hq, d), dtype=torch.bfloat16, device=q.device)
+    _check(_lib.pa_decode_noalloc(_ptr(out), _ptr(q), _token_stride(q, "q"), _ptr(k_cache),
+                                  _ptr(v_cache), _ptr(block_tables), block_tables.shape[1],
+                                  _ptr(context_lens), B, int(max_context_len), hq, hkv, d, bs, nb,
+                                  float(scale), int(partition_size), PA_BF16, _ptr(err_flag),
+                                  _stream()), "pa_decode_noalloc")
     return out
 
 
