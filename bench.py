@@ -375,12 +375,20 @@ def secondary(torch, args, timer, pk):
 
 
 def load_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch recorded from an ncu capture of this kernel and workload, if any."""
+    """DRAM bytes (read + write) per launch from an ncu capture of this kernel and
+    workload, or None when there is none or the kernel's source changed since."""
+    import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p))
-    return d.get(f"{kernel}:{workload}")
+    e = json.load(open(p)).get(f"{kernel}:{workload}")
+    if not e:
+        return None
+    src = os.path.join(ROOT, e["source"])
+    if not os.path.exists(src) or \
+            hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != e["source_sha256_16"]:
+        return None
+    return e["bytes"]
 
 
 # ------------------------------------------------------------ CPU oracle arm
