@@ -1,0 +1,107 @@
+"""Trace replay on the GPU checked against the oracle (``-m gpu``).
+
+A small trace (tiny pool, so preemption fires) is checked at every step and
+every layer: the oracle recomputes each sequence's slots from its block table,
+rebuilds the sequence's K/V history from the host record of which ring row
+last wrote each slot (CPU copies of the ring; nothing read back from the
+pool), and runs ``ref_prefill`` / ``ref_decode``.  The full 512-request trace
+is checked on sampled steps and layers.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_attention_35_b200.replay import Replay, ReplayConfig
+from tests.gpu_cases import TOL_MAX, TOL_MEAN
+from tests.problems import to_bits
+
+pytestmark = pytest.mark.gpu
+f64 = oracle.bf16_bits_to_f64
+
+
+def _history(rp, snap, block_table, length, layer, which):
+    """[length, Hkv, D] float64 K (or V) rows a sequence's positions hold after a step."""
+    c = rp.cfg
+    slots = oracle.ref_slot_mapping(block_table, range(length), c.block_size)
+    writer = snap[slots]
+    assert (writer[:, 0] >= 0).all(), "a position was never stored"
+    ring = rp.k_ring_cpu if which == "k" else rp.v_ring_cpu
+    rows = [to_bits(ring[rp.ring_index(int(st), layer)][int(rw)]) for st, rw in writer]
+    return f64(np.stack(rows))
+
+
+def check_sample(rp, step, layer, max_seqs=None):
+    c = rp.cfg
+    smp = rp.samples[(step, layer)]
+    snap = rp.snap[step]
+    md = smp["md"]
+    q_all = f64(to_bits(rp.q_ring_cpu[rp.ring_index(step, layer)]))
+    out = smp["out"].double().numpy()
+    nseq = len(smp["lens"])
+    idx = range(nseq) if max_seqs is None else np.linspace(0, nseq - 1, min(nseq, max_seqs)).astype(int)
+    errs = []
+    for j in idx:
+        bt = smp["block_tables"][j]
+        L = smp["lens"][j]
+        K = _history(rp, snap, bt, L, layer, "k")
+        V = _history(rp, snap, bt, L, layer, "v")
+        kp, vp = K[None], V[None]                     # one contiguous block holding the sequence
+        if smp["is_prefill"]:
+            a, b = int(md.cu_seqlens_q[j]), int(md.cu_seqlens_q[j + 1])
+            # the product's slots for the computed positions equal the oracle's
+            assert np.array_equal(md.slot_mapping[a:b],
+                                  oracle.ref_slot_mapping(bt, range(L - (b - a), L), c.block_size))
+            ref = oracle.ref_prefill(q_all[a:b], kp.reshape(1, L, c.num_kv_heads, c.head_dim),
+                                     vp.reshape(1, L, c.num_kv_heads, c.head_dim), [0, b - a], [0, L],
+                                     np.array([[0]]))
+            got = out[a:b]
+        else:
+            assert md.slot_mapping[j] == oracle.ref_slot_mapping(bt, [L - 1], c.block_size)[0]
+            assert md.context_lens[j] == L
+            ref = oracle.ref_decode(q_all[j:j + 1], kp.reshape(1, L, c.num_kv_heads, c.head_dim),
+                                    vp.reshape(1, L, c.num_kv_heads, c.head_dim), np.array([[0]]),
+                                    [L])
+            got = out[j:j + 1]
+        err = np.abs(got - ref)
+        assert np.isfinite(got).all()
+        errs.append((float(err.max()), float(err.mean())))
+    mx = max(e[0] for e in errs)
+    mean = float(np.mean([e[1] for e in errs]))
+    assert mx <= TOL_MAX and mean <= TOL_MEAN, (step, layer, mx, mean)
+
+
+def test_small_trace_every_step(cuda_device):
+    cfg = ReplayConfig(num_requests=14, prompt_lo=5, prompt_hi=70, output_lo=3, output_hi=40,
+                       max_num_seqs=6, max_num_batched_tokens=160, block_size=16, num_blocks=14,
+                       num_layers=2, num_q_heads=8, num_kv_heads=2, head_dim=128, ring=3, seed=4242,
+                       max_model_len=128)
+    rp = Replay(cfg, record="all")
+    st = rp.run()
+    assert st["finished"] == cfg.num_requests
+    assert st["preemptions"] > 0, "the tiny pool should force preemption"
+    assert st["prefill_steps"] > 0 and st["decode_steps"] > 0
+    for s in rp.requests:
+        assert s.num_completion_tokens == s.max_tokens
+    for (step, layer) in sorted(rp.samples):
+        check_sample(rp, step, layer)
+    rp.sched.block_manager.check_invariants([])
+    assert rp.sched.block_manager.num_free_blocks == cfg.num_blocks
+
+
+def test_full_trace_sampled(cuda_device):
+    """512 requests, prompt/output U[100,1024], 256 seqs, block 256, 768 blocks, 28 layers."""
+    cfg = ReplayConfig()
+    rp = Replay(cfg, record=True)
+    rp.sample_at = {(s, l) for s in (0, 3, 40, 400, 1100) for l in (0, cfg.num_layers - 1)}
+    st = rp.run()
+    assert st["finished"] == cfg.num_requests
+    assert st["preemptions"] > 0
+    checked = 0
+    for key in sorted(rp.samples):
+        check_sample(rp, *key, max_seqs=6)
+        checked += 1
+    assert checked >= 6
