@@ -17,6 +17,8 @@
 // prefill_tc.cu is the fast path for head_dim 128.
 
 #include <cmath>
+#include <cstdlib>
+#include <cstring>
 
 #include "pa_common.cuh"
 #include "pa_internal.h"
@@ -366,6 +368,17 @@ pa_status launch_prefill_mma(const PrefillArgs& a) {
   return launch_prefill_mma_d<64>(a, mk, mv, prm);
 }
 
-pa_status launch_prefill(const PrefillArgs& a) { return launch_prefill_mma(a); }
+pa_status launch_prefill_tc(const PrefillArgs& a);
+
+// head_dim 128 runs on the tcgen05 kernel; PA_PREFILL_PATH=mma selects the
+// mma.sync kernel instead (both are GPU kernels; the switch exists to compare them).
+pa_status launch_prefill(const PrefillArgs& a) {
+  static const bool force_mma = [] {
+    const char* e = getenv("PA_PREFILL_PATH");
+    return e && strcmp(e, "mma") == 0;
+  }();
+  if (a.d == 128 && !force_mma) return launch_prefill_tc(a);
+  return launch_prefill_mma(a);
+}
 
 }  // namespace pa
