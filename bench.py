@@ -374,6 +374,34 @@ def secondary(torch, args, timer, pk):
     return out
 
 
+def only(args):
+    """One secondary workload by itself (profiling aid); prints its JSON object."""
+    import torch
+    from paged_kv_attention_35_b200 import synth
+    from paged_kv_attention_35_b200.workloads import DecodeWorkload
+    pk = peaks()
+    timer = Timer(torch)
+    if args.only == "prefill":
+        w, store_ms, attn_ms = bench_prefill(torch, args.steps, args.warmup, timer)
+        tf = w.flops() / (attn_ms * 1e-3) / 1e12
+        res = {"workload": "prefix_prefill", "attn_ms": round(attn_ms, 4), "TFLOPs": round(tf, 1),
+               "frac_bf16_peak": round(tf / pk["bf16_tflops"], 4)}
+    elif args.only == "decode_gqa":
+        w = DecodeWorkload.from_spec(synth.WORKLOADS["gqa7b_decode"]).upload("cuda")
+        r = bench_decode(torch, w, args.steps, args.warmup, timer, partition=args.partition)
+        gbs = w.kv_bytes() / (r["decode_ms"] * 1e-3) / 1e9
+        res = {"workload": "gqa7b_decode", "decode_ms": round(r["decode_ms"], 4),
+               "decode_GBs": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4)}
+    elif args.only == "store":
+        nbytes, ms = bench_store_large(torch, args.steps, args.warmup, timer)
+        res = {"workload": "store_kvcache_65536", "ms": round(ms, 4),
+               "GBs": round(nbytes / (ms * 1e-3) / 1e9, 1)}
+    else:
+        from paged_kv_attention_35_b200.replay import run_replay_bench
+        res = run_replay_bench(torch, max_steps=args.replay_steps)
+    print(json.dumps(res), flush=True)
+
+
 def load_traffic(kernel: str, workload: str):
     """DRAM bytes (read + write) per launch from an ncu capture of this kernel and
     workload, or None when there is none or the kernel's source changed since."""
@@ -498,11 +526,15 @@ def main():
     ap.add_argument("--no-replay", action="store_true")
     ap.add_argument("--replay-steps", type=int, default=0)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--only", choices=["prefill", "decode_gqa", "store", "replay"], default=None,
+                    help="time one secondary workload alone (for profiling) and print its JSON")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         reference(args)
+    elif args.only:
+        only(args)
     else:
         ours(args)
 

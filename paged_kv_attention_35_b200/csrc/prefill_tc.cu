@@ -7,25 +7,27 @@
 // attends keys 0 .. k_len-q_len+j; prompts are batched by cumulative sequence
 // lengths ("Preparation before computation", same item).
 //
-// One CTA = 128 query rows of one (sequence, query head); 6 warps:
-//   warp 4      TMA producer: the Q tile once, then 128-key K and V tiles of
-//               the sequence (one box per physical block chunk, 128-byte
-//               swizzle) into a 2-stage ring; zeroes V rows of the last tile
-//               past the CTA's last visible key (stale rows may be NaN).
-//   warp 5      MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM S
-//               buffers (M=128, N=128, K=16 x 8), then O += P_j V_j into the
-//               TMEM O accumulator (A = P from shared memory, B = V MN-major);
-//               tcgen05.commit signals mbarriers.  S_{j+1} is issued before
-//               waiting for P_j, so QK^T of the next tile overlaps the softmax.
-//   warps 0-3   softmax, one thread per query row (TMEM lane): tcgen05.ld the
-//               S row, causal mask, online softmax in the log2 domain with a
-//               lazy rescale (the reference max moves only when it grows by
-//               more than 8, i.e. a factor 256), P as bf16 into shared memory
-//               (swizzled, K-major), O rescaled in TMEM when needed; epilogue
-//               O / l -> bf16 -> global.
-// TMEM: 512 columns (S0 | S1 | O | unused).  Shared memory: Q 32 KB, K and V
-// 2 x 32 KB each, P 32 KB.  Every wait is bounded; an abort winds all roles
-// down, drains the issued MMAs and frees TMEM.
+// One CTA = two consecutive 128-row query tiles (A, B) of one (sequence,
+// query head); 10 warps:
+//   warp 8      TMA producer: both Q tiles once, then 128-key K and V tiles of
+//               the sequence (one box per physical-block chunk, 128-byte
+//               swizzle) into a 3-slot ring (K_j, V_j, K_j+1, ...) shared by
+//               both tiles; zeroes V rows of the last tile past the CTA's last
+//               visible key (stale pool rows may hold NaN).
+//   warp 9      MMA issuer (one thread): S_t(j) = Q_t K_j^T into tile t's TMEM
+//               S buffer (M=128, N=128, K=16 x 8) and O_t += P_t(j) V_j into its
+//               TMEM O accumulator (A = P from shared memory, B = V MN-major),
+//               interleaving the tiles so one tile's softmax overlaps the other
+//               tile's MMAs; tcgen05.commit signals the mbarriers.
+//   warps 0-3 / 4-7   softmax of tile A / B, one thread per query row (TMEM
+//               lane): tcgen05.ld the S row, causal mask on diagonal tiles only,
+//               online softmax in the log2 domain with a lazy rescale (the
+//               reference max moves only when it grows by more than 8, a factor
+//               256), P as bf16 into shared memory (swizzled, K-major), O
+//               rescaled in TMEM when needed; epilogue O / l -> bf16 -> global.
+// TMEM: 512 columns (S_A | O_A | S_B | O_B).  Shared memory: Q 2 x 32 KB, P
+// 2 x 32 KB, K/V ring 3 x 32 KB.  Every wait is bounded; an abort winds all
+// roles down, drains the issued MMAs and frees TMEM.
 
 #include <cmath>
 
@@ -35,11 +37,12 @@
 
 namespace pa {
 
-constexpr int kTcRows = 128;     // query rows per CTA (MMA M)
-constexpr int kTcKeys = 128;     // keys per tile (MMA N of QK^T, K of PV)
-constexpr int kTcThreads = 192;
+constexpr int kTcRows = 128;     // query rows per tile (MMA M)
+constexpr int kTcKeys = 128;     // keys per KV tile (MMA N of QK^T, K of PV)
+constexpr int kTcThreads = 320;  // 2 softmax warpgroups + producer warp + MMA warp
 constexpr int kTile = 32768;     // one 128 x 128 bf16 operand: two 128 x 64 swizzled halves
 constexpr int kHalf = 16384;
+constexpr int kRing = 3;         // K/V ring slots (K_j, V_j, K_j+1, ... in turn)
 constexpr float kLazyRescale = 8.f;   // log2 of the largest un-rescaled growth (256x)
 
 struct PrefillTcParams {
@@ -73,92 +76,107 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
   }
 }
 
+// Barrier block in shared memory (after the operand buffers).
+struct TcBars {
+  uint64_t q_full;
+  uint64_t kv_full[kRing];
+  uint64_t kv_empty[kRing];
+  uint64_t s_full[2];      // per query tile (A, B)
+  uint64_t p_full[2];
+  uint64_t pv_done[2];
+  uint64_t vz_ready;
+  uint64_t drain;
+  uint32_t tmem;
+  int abort_flag;
+};
+
+// One CTA = two consecutive 128-row query tiles (A, B) of one (sequence, head).
+// The MMA thread interleaves them so that the softmax of one tile overlaps the
+// other tile's P V and next Q K^T on the tensor core:
+//   S_A(0) S_B(0) | PV_A(0) S_A(1) | PV_B(0) S_B(1) | PV_A(1) S_A(2) | ...
+// Both tiles read the same K/V tiles (the later tile needs at most one more).
 __global__ void __launch_bounds__(kTcThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const PrefillTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + kTile;              // [2 stages]
-  uint8_t* sV = sK + 2 * kTile;          // [2 stages]
-  uint8_t* sP = sV + 2 * kTile;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + kTile);
-  uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;           // [2]
-  uint64_t* v_full = bars + 3;           // [2]
-  uint64_t* kv_empty = bars + 5;         // [2]
-  uint64_t* s_full = bars + 7;           // [2]
-  uint64_t* s_free = bars + 9;           // [2]
-  uint64_t* p_full = bars + 11;
-  uint64_t* pv_done = bars + 12;
-  uint64_t* vz_ready = bars + 13;
-  uint64_t* drain = bars + 14;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 16);
+  uint8_t* sQ = smem;                     // [2 tiles]
+  uint8_t* sP = sQ + 2 * kTile;           // [2 tiles]
+  uint8_t* sKV = sP + 2 * kTile;          // [kRing slots]
+  TcBars* bar = reinterpret_cast<TcBars*>(sKV + kRing * kTile);
+  volatile int* abort_flag = &bar->abort_flag;
 
-  const int qtile = blockIdx.x, h = blockIdx.y, seq = blockIdx.z;
+  // longest pairs first: the last query tiles of a sequence see the most keys
+  const int pair = gridDim.x - 1 - blockIdx.x;
+  const int h = blockIdx.y, seq = blockIdx.z;
   const int kvh = h / p.group;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // sequence bounds
   const int cq0 = __ldg(p.cu_q + seq), cq1 = __ldg(p.cu_q + seq + 1);
   const int ck0 = __ldg(p.cu_k + seq), ck1 = __ldg(p.cu_k + seq + 1);
   const int q_start = cq0, q_len = cq1 - cq0, k_len = ck1 - ck0;
   if (!(cq0 >= 0 && q_len >= 0 && cq1 <= p.total_q && k_len >= q_len &&
         q_len <= p.max_seqlen_q && k_len <= p.max_seqlen_k && k_len <= p.max_blocks * p.block_size)) {
-    if (threadIdx.x == 0 && qtile == 0 && h == 0) raise_flag(p.err_flag, PA_FLAG_LEN_OOB);
+    if (threadIdx.x == 0 && blockIdx.x == 0 && h == 0) raise_flag(p.err_flag, PA_FLAG_LEN_OOB);
     return;
   }
-  const int q0 = qtile * kTcRows;
-  if (q0 >= q_len) return;
+  const int q0A = pair * 2 * kTcRows;
+  if (q0A >= q_len) return;
+  const int q0B = q0A + kTcRows;
+  const bool hasB = q0B < q_len;
   const int cached = k_len - q_len;
-  const int kv_end = min(k_len, cached + min(q_len, q0 + kTcRows));   // keys any row can see
-  const int n = (kv_end + kTcKeys - 1) / kTcKeys;
+  const int kv_endA = min(k_len, cached + min(q_len, q0A + kTcRows));
+  const int kv_endB = hasB ? min(k_len, cached + min(q_len, q0B + kTcRows)) : 0;
+  const int nA = (kv_endA + kTcKeys - 1) / kTcKeys;
+  const int nB = (kv_endB + kTcKeys - 1) / kTcKeys;
+  const int kv_end = max(kv_endA, kv_endB);
+  const int n = max(nA, nB);
   const int last_valid = kv_end - (n - 1) * kTcKeys;
   const bool zero_tail = last_valid < kTcKeys;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
-      mbar_init(&s_full[s], 1);
-      mbar_init(&s_free[s], 4);
+    mbar_init(&bar->q_full, 1);
+    for (int s = 0; s < kRing; ++s) {
+      mbar_init(&bar->kv_full[s], 1);
+      mbar_init(&bar->kv_empty[s], 1);
     }
-    mbar_init(p_full, 4);
-    mbar_init(pv_done, 1);
-    mbar_init(vz_ready, 1);
-    mbar_init(drain, 1);
-    *abort_flag = 0;
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bar->s_full[t], 1);
+      mbar_init(&bar->p_full[t], 4);
+      mbar_init(&bar->pv_done[t], 1);
+    }
+    mbar_init(&bar->vz_ready, 1);
+    mbar_init(&bar->drain, 1);
+    bar->abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
-    tc::tmem_alloc(tmem_slot, 512);
+  if (warp == 9) {
+    tc::tmem_alloc(&bar->tmem, 512);
     tc::tmem_relinquish();
   }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem;               // S buffers: columns [0,128) and [128,256)
-  const uint32_t tO = tmem + 256;         // O accumulator: columns [256,384)
+  const uint32_t tmem = bar->tmem;        // tile t: S at columns [256t, 256t+128), O at +128
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(q_full, kTile);
-      tma_load_3d(sQ, &tmQ, q_full, 0, h, q_start + q0);
-      tma_load_3d(sQ + kHalf, &tmQ, q_full, 64, h, q_start + q0);
+      mbar_arrive_expect_tx(&bar->q_full, hasB ? 2 * kTile : kTile);
+      tma_load_3d(sQ, &tmQ, &bar->q_full, 0, h, q_start + q0A);
+      tma_load_3d(sQ + kHalf, &tmQ, &bar->q_full, 64, h, q_start + q0A);
+      if (hasB) {
+        tma_load_3d(sQ + kTile, &tmQ, &bar->q_full, 0, h, q_start + q0B);
+        tma_load_3d(sQ + kTile + kHalf, &tmQ, &bar->q_full, 64, h, q_start + q0B);
+      }
       const int32_t* bt = p.block_tables + (int64_t)seq * p.max_blocks;
       const int box = p.box_rows;
+      int i = 0;
       for (int j = 0; j < n; ++j) {
-        const int st = j & 1;
-        if (j >= 2 && !tc_wait(&kv_empty[st], ((j >> 1) - 1) & 1, abort_flag, p.err_flag)) break;
         const int t0 = j * kTcKeys;
         const int nbox = (min(kTcKeys, kv_end - t0) + box - 1) / box;
         const uint32_t bytes = (uint32_t)(nbox * box * 128 * 2);
@@ -173,160 +191,192 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             rows[b] = bid * p.block_size + (t & (p.block_size - 1));
           }
         }
-        mbar_arrive_expect_tx(&k_full[st], bytes);
-        for (int b = 0; b < nbox; ++b) {
-          uint8_t* dst = sK + st * kTile + b * box * 128;
-          tma_load_3d(dst, &tmK, &k_full[st], 0, kvh, rows[b]);
-          tma_load_3d(dst + kHalf, &tmK, &k_full[st], 64, kvh, rows[b]);
+        bool ok = true;
+        for (int kv = 0; kv < 2; ++kv, ++i) {
+          const int slot = i % kRing;
+          if (i >= kRing &&
+              !tc_wait(&bar->kv_empty[slot], ((i / kRing) - 1) & 1, abort_flag, p.err_flag)) {
+            ok = false;
+            break;
+          }
+          const CUtensorMap* map = kv ? &tmV : &tmK;
+          mbar_arrive_expect_tx(&bar->kv_full[slot], bytes);
+          for (int b = 0; b < nbox; ++b) {
+            uint8_t* dst = sKV + slot * kTile + b * box * 128;
+            tma_load_3d(dst, map, &bar->kv_full[slot], 0, kvh, rows[b]);
+            tma_load_3d(dst + kHalf, map, &bar->kv_full[slot], 64, kvh, rows[b]);
+          }
         }
-        mbar_arrive_expect_tx(&v_full[st], bytes);
-        for (int b = 0; b < nbox; ++b) {
-          uint8_t* dst = sV + st * kTile + b * box * 128;
-          tma_load_3d(dst, &tmV, &v_full[st], 0, kvh, rows[b]);
-          tma_load_3d(dst + kHalf, &tmV, &v_full[st], 64, kvh, rows[b]);
-        }
+        if (!ok) break;
       }
     }
     __syncwarp();
     if (zero_tail) {
-      const int j = n - 1, st = j & 1;
-      if (tc_wait(&v_full[st], (j >> 1) & 1, abort_flag, p.err_flag)) {
+      const int iv = 2 * (n - 1) + 1, slot = iv % kRing;
+      if (tc_wait(&bar->kv_full[slot], (iv / kRing) & 1, abort_flag, p.err_flag)) {
         const int nrow = kTcKeys - last_valid;
-        for (int i = lane; i < nrow * 16; i += 32) {
-          const int hf = i / (nrow * 8);
-          const int rr = (i / 8) % nrow;
-          *reinterpret_cast<uint4*>(sV + st * kTile + hf * kHalf + (last_valid + rr) * 128 +
-                                    (i & 7) * 16) = make_uint4(0, 0, 0, 0);
+        for (int t = lane; t < nrow * 16; t += 32) {
+          const int hf = t / (nrow * 8);
+          const int rr = (t / 8) % nrow;
+          *reinterpret_cast<uint4*>(sKV + slot * kTile + hf * kHalf + (last_valid + rr) * 128 +
+                                    (t & 7) * 16) = make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(vz_ready);
+      if (lane == 0) mbar_arrive(&bar->vz_ready);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = tc::idesc_bf16(kTcRows, kTcKeys, false, false);
       constexpr uint32_t idO = tc::idesc_bf16(kTcRows, 128, false, true);
-      const uint32_t aQ = smem_u32(sQ), aP = smem_u32(sP);
-      bool ok = tc_wait(q_full, 0, abort_flag, p.err_flag);
-      auto issue_s = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!tc_wait(&k_full[st], (j >> 1) & 1, abort_flag, p.err_flag)) return false;
-        if (j >= 2 && !tc_wait(&s_free[st], ((j >> 1) - 1) & 1, abort_flag, p.err_flag)) return false;
-        tc::fence_after_sync();
-        const uint32_t aK = smem_u32(sK + st * kTile);
+      const int ntile[2] = {nA, nB};
+      auto issue_s = [&](int t, int j) {          // S_t(j) = Q_t K_j^T
+        const int slot = (2 * j) % kRing;
+        const uint32_t aQ = smem_u32(sQ + t * kTile), aK = smem_u32(sKV + slot * kTile);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
-          tc::mma_ss(tS + st * 128, tc::sdesc_sw128(aQ + o, 16, 1024),
+          tc::mma_ss(tmem + 256 * t, tc::sdesc_sw128(aQ + o, 16, 1024),
                      tc::sdesc_sw128(aK + o, 16, 1024), idS, ks > 0);
         }
-        tc::commit(&s_full[st]);
-        return true;
+        tc::commit(&bar->s_full[t]);
       };
-      if (ok) ok = issue_s(0);
-      for (int j = 0; ok && j < n; ++j) {
-        if (j + 1 < n && !issue_s(j + 1)) break;
-        if (!tc_wait(p_full, j & 1, abort_flag, p.err_flag)) break;
-        const bool vz = zero_tail && j == n - 1;
-        if (!tc_wait(vz ? vz_ready : &v_full[j & 1], vz ? 0u : (uint32_t)((j >> 1) & 1), abort_flag,
-                     p.err_flag))
-          break;
+      auto wait_k = [&](int j) {
+        const int i = 2 * j;
+        return tc_wait(&bar->kv_full[i % kRing], (i / kRing) & 1, abort_flag, p.err_flag);
+      };
+      bool ok = tc_wait(&bar->q_full, 0, abort_flag, p.err_flag) && wait_k(0);
+      if (ok) {
         tc::fence_after_sync();
-        const uint32_t aV = smem_u32(sV + (j & 1) * kTile);
+        issue_s(0, 0);
+        if (nB > 0) issue_s(1, 0);
+        tc::commit(&bar->kv_empty[0]);          // K_0 consumed by both tiles
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        const int iv = 2 * j + 1, vslot = iv % kRing;
+        const bool vz = zero_tail && j == n - 1;
+        bool v_ready = false, k_next = false;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j >= ntile[t]) continue;
+          if (!tc_wait(&bar->p_full[t], j & 1, abort_flag, p.err_flag)) { ok = false; break; }
+          if (!v_ready) {
+            if (!tc_wait(vz ? &bar->vz_ready : &bar->kv_full[vslot], vz ? 0u : (uint32_t)((iv / kRing) & 1),
+                         abort_flag, p.err_flag)) { ok = false; break; }
+            v_ready = true;
+          }
+          tc::fence_after_sync();
+          const uint32_t aP = smem_u32(sP + t * kTile), aV = smem_u32(sKV + vslot * kTile);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t oa = (ks >> 2) * kHalf + (ks & 3) * 32;
-          tc::mma_ss(tO, tc::sdesc_sw128(aP + oa, 16, 1024),
-                     tc::sdesc_sw128(aV + ks * 2048, kHalf, 1024), idO, (j > 0 || ks > 0));
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t oa = (ks >> 2) * kHalf + (ks & 3) * 32;
+            tc::mma_ss(tmem + 256 * t + 128, tc::sdesc_sw128(aP + oa, 16, 1024),
+                       tc::sdesc_sw128(aV + ks * 2048, kHalf, 1024), idO, (j > 0 || ks > 0));
+          }
+          tc::commit(&bar->pv_done[t]);
+          if (j + 1 < ntile[t]) {
+            if (!k_next) {
+              if (!wait_k(j + 1)) { ok = false; break; }
+              k_next = true;
+              tc::fence_after_sync();
+            }
+            issue_s(t, j + 1);
+          }
         }
-        tc::commit(pv_done);
-        tc::commit(&kv_empty[j & 1]);
+        if (!ok) break;
+        tc::commit(&bar->kv_empty[vslot]);                 // V_j consumed
+        if (j + 1 < n) tc::commit(&bar->kv_empty[(2 * (j + 1)) % kRing]);   // K_j+1 consumed
       }
       // every issued MMA finishes before TMEM is released
-      tc::commit(drain);
-      mbar_wait(drain, 0);
+      tc::commit(&bar->drain);
+      mbar_wait(&bar->drain, 0);
     }
   } else {
-    // ------------------------------------------------------------ softmax
-    const int r = threadIdx.x;                         // query row within the tile = TMEM lane
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const int limit = min(cached + q0 + r, k_len - 1);  // last visible key of this row
+    // ------------------------------------------------------------ softmax (warpgroup t = tile)
+    const int t = warp >> 2;                       // 0: tile A, 1: tile B
+    const int r = threadIdx.x & 127;               // row within the tile = TMEM lane
+    const int nt = t ? nB : nA;
+    const int q0 = t ? q0B : q0A;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + 256 * t + lane_off, tO = tS + 128;
+    const int limit = min(cached + q0 + r, k_len - 1);   // last visible key of this row
+    const float sl2 = p.scale_log2;
+    uint8_t* myP = sP + t * kTile;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    uint32_t sv[kTcKeys];
-    for (int j = 0; j < n; ++j) {
-      const int b = j & 1;
-      if (!tc_wait(&s_full[b], (j >> 1) & 1, abort_flag, p.err_flag)) { ok = false; break; }
+    float sv[kTcKeys];
+    for (int j = 0; j < nt; ++j) {
+      if (!tc_wait(&bar->s_full[t], j & 1, abort_flag, p.err_flag)) { ok = false; break; }
       tc::fence_after_sync();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tc::ld32(tS + lane_off + b * 128 + c * 32, sv + c * 32);
+      for (int c = 0; c < 4; ++c) tc::ld32(tS + c * 32, reinterpret_cast<uint32_t*>(sv) + c * 32);
       tc::wait_ld();
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[b]);
       const int t0 = j * kTcKeys;
       float mx = -INFINITY;
+      if (t0 + kTcKeys - 1 > limit) {              // diagonal / tail tile: mask
 #pragma unroll
-      for (int i = 0; i < kTcKeys; ++i) {
-        const float s = (t0 + i <= limit) ? __uint_as_float(sv[i]) * p.scale_log2 : -INFINITY;
-        sv[i] = __float_as_uint(s);
-        mx = fmaxf(mx, s);
+        for (int i = 0; i < kTcKeys; ++i) {
+          sv[i] = (t0 + i <= limit) ? sv[i] : -INFINITY;
+          mx = fmaxf(mx, sv[i]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < kTcKeys; ++i) mx = fmaxf(mx, sv[i]);
       }
+      mx *= sl2;                                   // scale > 0: max commutes with it
       float alpha = 1.f;
       bool resc = false;
       if (m_ref == -INFINITY) {
-        m_ref = mx;                                    // first tile with a visible key
+        m_ref = mx;
       } else if (mx > m_ref + kLazyRescale) {
         alpha = fast_exp2(m_ref - mx);
         m_ref = mx;
         resc = true;
         l *= alpha;
       }
-      const float mref = m_ref == -INFINITY ? 0.f : m_ref;
+      const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
       float rs = 0.f;
 #pragma unroll
       for (int i = 0; i < kTcKeys; ++i) {
-        const float e = fast_exp2(__uint_as_float(sv[i]) - mref);
-        rs += e;
-        sv[i] = __float_as_uint(e);
+        sv[i] = fast_exp2(fmaf(sv[i], sl2, neg_m));
+        rs += sv[i];
       }
       l += rs;
-      // PV_{j-1} must be done before P is overwritten and O is rescaled
-      if (j > 0 && !tc_wait(pv_done, (j - 1) & 1, abort_flag, p.err_flag)) { ok = false; break; }
+      // P V of the previous tile must be done before P is overwritten and O rescaled
+      if (j > 0 && !tc_wait(&bar->pv_done[t], (j - 1) & 1, abort_flag, p.err_flag)) { ok = false; break; }
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
           const int i0 = hf * 64 + ch * 8;
           uint4 v;
-          v.x = pack_bf16(__uint_as_float(sv[i0 + 0]), __uint_as_float(sv[i0 + 1]));
-          v.y = pack_bf16(__uint_as_float(sv[i0 + 2]), __uint_as_float(sv[i0 + 3]));
-          v.z = pack_bf16(__uint_as_float(sv[i0 + 4]), __uint_as_float(sv[i0 + 5]));
-          v.w = pack_bf16(__uint_as_float(sv[i0 + 6]), __uint_as_float(sv[i0 + 7]));
-          *reinterpret_cast<uint4*>(sP + hf * kHalf + sw128(r, ch)) = v;
+          v.x = pack_bf16(sv[i0 + 0], sv[i0 + 1]);
+          v.y = pack_bf16(sv[i0 + 2], sv[i0 + 3]);
+          v.z = pack_bf16(sv[i0 + 4], sv[i0 + 5]);
+          v.w = pack_bf16(sv[i0 + 6], sv[i0 + 7]);
+          *reinterpret_cast<uint4*>(myP + hf * kHalf + sw128(r, ch)) = v;
         }
       if (__any_sync(0xffffffffu, resc)) {
         tc::fence_after_sync();
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t ov[32];
-          tc::ld32(tO + lane_off + c * 32, ov);
+          tc::ld32(tO + c * 32, ov);
           tc::wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-          tc::st32(tO + lane_off + c * 32, ov);
+          tc::st32(tO + c * 32, ov);
         }
         tc::wait_st();
       }
-      fence_proxy_async_smem();                        // P visible to the tensor core
+      fence_proxy_async_smem();                    // P visible to the tensor core
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&bar->p_full[t]);
     }
     // epilogue: O / l -> bf16
-    if (ok && tc_wait(pv_done, (n - 1) & 1, abort_flag, p.err_flag)) {
+    if (nt > 0 && ok && tc_wait(&bar->pv_done[t], (nt - 1) & 1, abort_flag, p.err_flag)) {
       tc::fence_after_sync();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const bool store = q0 + r < q_len;
@@ -334,7 +384,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t ov[32];
-        tc::ld32(tO + lane_off + c * 32, ov);
+        tc::ld32(tO + c * 32, ov);
         tc::wait_ld();
         if (store) {
 #pragma unroll
@@ -353,7 +403,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, 512);
   }
@@ -387,7 +437,7 @@ pa_status launch_prefill_tc(const PrefillArgs& a) {
   prm.total_q = a.total_q;
   prm.scale_log2 = a.scale * 1.4426950408889634f;
   prm.err_flag = a.err_flag;
-  const size_t smem = 6 * (size_t)kTile + 1024 + 256;
+  const size_t smem = (4 + kRing) * (size_t)kTile + 1024 + sizeof(TcBars);
   static bool attr_done = false;
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel,
@@ -396,7 +446,7 @@ pa_status launch_prefill_tc(const PrefillArgs& a) {
     attr_done = true;
   }
   if (a.hq > 65535) return fail(PA_ERR_UNSUPPORTED, "too many heads");
-  dim3 grid((a.max_seqlen_q + kTcRows - 1) / kTcRows, a.hq, a.num_seqs);
+  dim3 grid((a.max_seqlen_q + 2 * kTcRows - 1) / (2 * kTcRows), a.hq, a.num_seqs);
   prefill_tc_kernel<<<grid, kTcThreads, smem, a.stream>>>(mq, mk, mv, prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "prefill_tc launch");
