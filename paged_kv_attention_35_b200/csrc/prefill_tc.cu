@@ -11,23 +11,26 @@
 // query head); 10 warps:
 //   warp 8      TMA producer: both Q tiles once, then 128-key K and V tiles of
 //               the sequence (one box per physical-block chunk, 128-byte
-//               swizzle) into a 3-slot ring (K_j, V_j, K_j+1, ...) shared by
+//               swizzle) into a 5-slot ring (K_j, V_j, K_j+1, ...) shared by
 //               both tiles; zeroes V rows of the last tile past the CTA's last
 //               visible key (stale pool rows may hold NaN).
 //   warp 9      MMA issuer (one thread): S_t(j) = Q_t K_j^T into tile t's TMEM
 //               S buffer (M=128, N=128, K=16 x 8) and O_t += P_t(j) V_j into its
-//               TMEM O accumulator (A = P from shared memory, B = V MN-major),
+//               TMEM O accumulator (A = P read from TMEM, B = V MN-major),
 //               interleaving the tiles so one tile's softmax overlaps the other
 //               tile's MMAs; tcgen05.commit signals the mbarriers.
 //   warps 0-3 / 4-7   softmax of tile A / B, one thread per query row (TMEM
 //               lane): tcgen05.ld the S row, causal mask on diagonal tiles only,
 //               online softmax in the log2 domain with a lazy rescale (the
 //               reference max moves only when it grows by more than 8, a factor
-//               256), P as bf16 into shared memory (swizzled, K-major), O
-//               rescaled in TMEM when needed; epilogue O / l -> bf16 -> global.
-// TMEM: 512 columns (S_A | O_A | S_B | O_B).  Shared memory: Q 2 x 32 KB, P
-// 2 x 32 KB, K/V ring 3 x 32 KB.  Every wait is bounded; an abort winds all
-// roles down, drains the issued MMAs and frees TMEM.
+//               256), P as bf16 pairs written back over the S columns it came
+//               from (tcgen05.st), O rescaled in TMEM when needed; epilogue
+//               O / l -> bf16 -> global.
+// TMEM: 512 columns (S_A/P_A | O_A | S_B/P_B | O_B).  The MMA thread issues
+// P V of a tile before that tile's next Q K^T, and tcgen05 MMAs of one thread
+// run in issue order, so the next S never overwrites P before P V has read it.
+// Shared memory: Q 2 x 32 KB, K/V ring 5 x 32 KB.  Every wait is bounded; an
+// abort winds all roles down, drains the issued MMAs and frees TMEM.
 
 #include <cmath>
 
@@ -42,7 +45,7 @@ constexpr int kTcKeys = 128;     // keys per KV tile (MMA N of QK^T, K of PV)
 constexpr int kTcThreads = 320;  // 2 softmax warpgroups + producer warp + MMA warp
 constexpr int kTile = 32768;     // one 128 x 128 bf16 operand: two 128 x 64 swizzled halves
 constexpr int kHalf = 16384;
-constexpr int kRing = 3;         // K/V ring slots (K_j, V_j, K_j+1, ... in turn)
+constexpr int kRing = 5;         // K/V ring slots (K_j, V_j, K_j+1, ... in turn)
 constexpr float kLazyRescale = 8.f;   // log2 of the largest un-rescaled growth (256x)
 
 struct PrefillTcParams {
@@ -102,8 +105,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sQ = smem;                     // [2 tiles]
-  uint8_t* sP = sQ + 2 * kTile;           // [2 tiles]
-  uint8_t* sKV = sP + 2 * kTile;          // [kRing slots]
+  uint8_t* sKV = sQ + 2 * kTile;          // [kRing slots]
   TcBars* bar = reinterpret_cast<TcBars*>(sKV + kRing * kTile);
   volatile int* abort_flag = &bar->abort_flag;
 
@@ -158,7 +160,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  const uint32_t tmem = bar->tmem;        // tile t: S at columns [256t, 256t+128), O at +128
+  // tile t: S at TMEM columns [256t, 256t+128) with P (bf16 pairs) over its first
+  // 64 columns once S has been read; O at [256t+128, 256t+256)
+  const uint32_t tmem = bar->tmem;
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
@@ -267,13 +271,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             v_ready = true;
           }
           tc::fence_after_sync();
-          const uint32_t aP = smem_u32(sP + t * kTile), aV = smem_u32(sKV + vslot * kTile);
+          const uint32_t aV = smem_u32(sKV + vslot * kTile);
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t oa = (ks >> 2) * kHalf + (ks & 3) * 32;
-            tc::mma_ss(tmem + 256 * t + 128, tc::sdesc_sw128(aP + oa, 16, 1024),
+          for (int ks = 0; ks < 8; ++ks)
+            tc::mma_ts(tmem + 256 * t + 128, tmem + 256 * t + ks * 8,
                        tc::sdesc_sw128(aV + ks * 2048, kHalf, 1024), idO, (j > 0 || ks > 0));
-          }
           tc::commit(&bar->pv_done[t]);
           if (j + 1 < ntile[t]) {
             if (!k_next) {
@@ -302,29 +304,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t tS = tmem + 256 * t + lane_off, tO = tS + 128;
     const int limit = min(cached + q0 + r, k_len - 1);   // last visible key of this row
     const float sl2 = p.scale_log2;
-    uint8_t* myP = sP + t * kTile;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     float sv[kTcKeys];
     for (int j = 0; j < nt; ++j) {
+      // S_t(j) complete implies every earlier MMA of this CTA -- P V of tile j-1
+      // included -- is complete: O may be rescaled and the S/P columns reused.
       if (!tc_wait(&bar->s_full[t], j & 1, abort_flag, p.err_flag)) { ok = false; break; }
       tc::fence_after_sync();
 #pragma unroll
       for (int c = 0; c < 4; ++c) tc::ld32(tS + c * 32, reinterpret_cast<uint32_t*>(sv) + c * 32);
       tc::wait_ld();
       const int t0 = j * kTcKeys;
-      float mx = -INFINITY;
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (t0 + kTcKeys - 1 > limit) {              // diagonal / tail tile: mask
 #pragma unroll
         for (int i = 0; i < kTcKeys; ++i) {
           sv[i] = (t0 + i <= limit) ? sv[i] : -INFINITY;
-          mx = fmaxf(mx, sv[i]);
+          mx4[i & 3] = fmaxf(mx4[i & 3], sv[i]);
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < kTcKeys; ++i) mx = fmaxf(mx, sv[i]);
+        for (int i = 0; i < kTcKeys; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], sv[i]);
       }
-      mx *= sl2;                                   // scale > 0: max commutes with it
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;  // scale > 0
       float alpha = 1.f;
       bool resc = false;
       if (m_ref == -INFINITY) {
@@ -336,29 +339,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         l *= alpha;
       }
       const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
-      float rs = 0.f;
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[kTcKeys / 2];
 #pragma unroll
-      for (int i = 0; i < kTcKeys; ++i) {
-        sv[i] = fast_exp2(fmaf(sv[i], sl2, neg_m));
-        rs += sv[i];
+      for (int i = 0; i < kTcKeys; i += 2) {
+        const float e0 = fast_exp2(fmaf(sv[i], sl2, neg_m));
+        const float e1 = fast_exp2(fmaf(sv[i + 1], sl2, neg_m));
+        rs4[(i >> 1) & 3] += e0 + e1;
+        pk[i >> 1] = pack_bf16(e0, e1);
       }
-      l += rs;
-      // P V of the previous tile must be done before P is overwritten and O rescaled
-      if (j > 0 && !tc_wait(&bar->pv_done[t], (j - 1) & 1, abort_flag, p.err_flag)) { ok = false; break; }
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const int i0 = hf * 64 + ch * 8;
-          uint4 v;
-          v.x = pack_bf16(sv[i0 + 0], sv[i0 + 1]);
-          v.y = pack_bf16(sv[i0 + 2], sv[i0 + 3]);
-          v.z = pack_bf16(sv[i0 + 4], sv[i0 + 5]);
-          v.w = pack_bf16(sv[i0 + 6], sv[i0 + 7]);
-          *reinterpret_cast<uint4*>(myP + hf * kHalf + sw128(r, ch)) = v;
-        }
+      l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+      tc::st32(tS, pk);                            // P over the first 64 S columns
+      tc::st32(tS + 32, pk + 32);
       if (__any_sync(0xffffffffu, resc)) {
-        tc::fence_after_sync();
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t ov[32];
@@ -368,9 +361,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
           tc::st32(tO + c * 32, ov);
         }
-        tc::wait_st();
       }
-      fence_proxy_async_smem();                    // P visible to the tensor core
+      tc::wait_st();
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar->p_full[t]);
@@ -437,7 +429,7 @@ pa_status launch_prefill_tc(const PrefillArgs& a) {
   prm.total_q = a.total_q;
   prm.scale_log2 = a.scale * 1.4426950408889634f;
   prm.err_flag = a.err_flag;
-  const size_t smem = (4 + kRing) * (size_t)kTile + 1024 + sizeof(TcBars);
+  const size_t smem = (2 + kRing) * (size_t)kTile + 1024 + sizeof(TcBars);
   static bool attr_done = false;
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel,

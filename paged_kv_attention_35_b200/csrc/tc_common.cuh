@@ -115,3 +115,19 @@ __device__ __forceinline__ void wait_st() { asm volatile("tcgen05.wait::st.sync.
 
 }  // namespace tc
 }  // namespace pa
+
+namespace pa {
+namespace tc {
+// D[tmem] (+)= A[tmem] * B[smem]: A (M x 16 bf16) is read from TMEM, lane =
+// row, each 32-bit column holding two consecutive K elements (low half first).
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+}  // namespace tc
+}  // namespace pa
