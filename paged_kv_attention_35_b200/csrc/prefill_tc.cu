@@ -79,6 +79,53 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
   }
 }
 
+// 2^x on the FMA pipe, for a share of the softmax exponentials so the MUFU
+// unit is not the only one computing them (x <= 8 here; results below 2^-125
+// are returned as 0).  Cody-Waite split x = n + f, n = floor(x), f in [0, 1);
+// 2^f from a degree-3 minimax polynomial fitted (Remez exchange, relative
+// error) on [0, 1): max relative error 7.5e-5, far below bf16's half-ulp
+// (2^-9) -- P is rounded to bf16 right after; 2^n is added to the exponent.
+__device__ __forceinline__ float exp2_poly(float x) {
+  const float xc = fmaxf(x, -125.f);
+  const float n = floorf(xc);
+  const float f = xc - n;
+  float q = fmaf(0.07802452264047931f, f, 0.22606715542748335f);
+  q = fmaf(q, f, 0.6958335404947529f);
+  q = fmaf(q, f, 0.9999252185627155f);
+  const float r = __int_as_float(__float_as_int(q) + (static_cast<int>(n) << 23));
+  return x < -125.f ? 0.f : r;
+}
+
+// Packed / 3-input fp32 arithmetic of sm_100 (halves the softmax's issue slots).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f32x2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+constexpr int kBtCache = 256;    // block-table entries staged in shared memory
+#ifndef PA_EXP_POLY_OF_8
+#define PA_EXP_POLY_OF_8 0         // exponential pairs out of every 8 computed by exp2_poly
+#endif
+
 // Barrier block in shared memory (after the operand buffers).
 struct TcBars {
   uint64_t q_full;
@@ -91,6 +138,7 @@ struct TcBars {
   uint64_t drain;
   uint32_t tmem;
   int abort_flag;
+  int bt[kBtCache];        // the sequence's first block-table entries
 };
 
 // One CTA = two consecutive 128-row query tiles (A, B) of one (sequence, head).
@@ -109,8 +157,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   TcBars* bar = reinterpret_cast<TcBars*>(sKV + kRing * kTile);
   volatile int* abort_flag = &bar->abort_flag;
 
-  // longest pairs first: the last query tiles of a sequence see the most keys
-  const int pair = gridDim.x - 1 - blockIdx.x;
+  // pair 0 = the sequence's last two query tiles (they see the most keys), so
+  // launch order is longest first and every CTA but possibly a sequence's
+  // first carries two tiles; tile A is the later one of the pair.
+  const int pp = blockIdx.x;
   const int h = blockIdx.y, seq = blockIdx.z;
   const int kvh = h / p.group;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -123,10 +173,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (threadIdx.x == 0 && blockIdx.x == 0 && h == 0) raise_flag(p.err_flag, PA_FLAG_LEN_OOB);
     return;
   }
-  const int q0A = pair * 2 * kTcRows;
-  if (q0A >= q_len) return;
-  const int q0B = q0A + kTcRows;
-  const bool hasB = q0B < q_len;
+  const int T = (q_len + kTcRows - 1) / kTcRows;   // query tiles of the sequence
+#ifdef PA_PAIR_FROM_START
+  const int tile_a = 2 * (gridDim.x - 1 - pp), tile_b = tile_a + 1;
+  if (tile_a >= T) return;
+  const bool hasB = tile_b < T;
+#else
+  if (2 * pp >= T) return;
+  const int tile_a = T - 1 - 2 * pp, tile_b = tile_a - 1;
+  const bool hasB = tile_b >= 0;
+#endif
+  const int q0A = tile_a * kTcRows;
+  const int q0B = hasB ? tile_b * kTcRows : 0;
   const int cached = k_len - q_len;
   const int kv_endA = min(k_len, cached + min(q_len, q0A + kTcRows));
   const int kv_endB = hasB ? min(k_len, cached + min(q_len, q0B + kTcRows)) : 0;
@@ -136,8 +194,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int n = max(nA, nB);
   const int last_valid = kv_end - (n - 1) * kTcKeys;
   const bool zero_tail = last_valid < kTcKeys;
+  const int32_t* bt = p.block_tables + (int64_t)seq * p.max_blocks;
 
-  if (threadIdx.x == 0) {
+  if (warp == 8 && lane == 0) {
+    // the producer thread sets up the barriers and starts the Q loads at once
     mbar_init(&bar->q_full, 1);
     for (int s = 0; s < kRing; ++s) {
       mbar_init(&bar->kv_full[s], 1);
@@ -152,6 +212,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     mbar_init(&bar->drain, 1);
     bar->abort_flag = 0;
     fence_barrier_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    mbar_arrive_expect_tx(&bar->q_full, hasB ? 2 * kTile : kTile);
+    tma_load_3d(sQ, &tmQ, &bar->q_full, 0, h, q_start + q0A);
+    tma_load_3d(sQ + kHalf, &tmQ, &bar->q_full, 64, h, q_start + q0A);
+    if (hasB) {
+      tma_load_3d(sQ + kTile, &tmQ, &bar->q_full, 0, h, q_start + q0B);
+      tma_load_3d(sQ + kTile + kHalf, &tmQ, &bar->q_full, 64, h, q_start + q0B);
+    }
+  }
+  if (warp == 8) {
+    // stage the block-table entries this CTA reads (all lanes, one round trip)
+    const int nblk = min((kv_end + p.block_size - 1) >> p.log2_bs, kBtCache);
+    for (int i = lane; i < nblk; i += 32) bar->bt[i] = __ldg(bt + i);
   }
   if (warp == 9) {
     tc::tmem_alloc(&bar->tmem, 512);
@@ -167,17 +242,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(&bar->q_full, hasB ? 2 * kTile : kTile);
-      tma_load_3d(sQ, &tmQ, &bar->q_full, 0, h, q_start + q0A);
-      tma_load_3d(sQ + kHalf, &tmQ, &bar->q_full, 64, h, q_start + q0A);
-      if (hasB) {
-        tma_load_3d(sQ + kTile, &tmQ, &bar->q_full, 0, h, q_start + q0B);
-        tma_load_3d(sQ + kTile + kHalf, &tmQ, &bar->q_full, 64, h, q_start + q0B);
-      }
-      const int32_t* bt = p.block_tables + (int64_t)seq * p.max_blocks;
       const int box = p.box_rows;
       int i = 0;
       for (int j = 0; j < n; ++j) {
@@ -187,7 +251,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         int rows[kTcKeys / 16];
         for (int b = 0; b < nbox; ++b) {
           const int t = t0 + b * box;
-          const int bid = __ldg(bt + (t >> p.log2_bs));
+          const int lb = t >> p.log2_bs;
+          const int bid = lb < kBtCache ? bar->bt[lb] : __ldg(bt + lb);
           if (bid < 0 || bid >= p.num_blocks) {
             raise_flag(p.err_flag, PA_FLAG_BLOCK_OOB);
             rows[b] = p.num_slots;                 // past the pool: TMA fills zeros
@@ -316,18 +381,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int c = 0; c < 4; ++c) tc::ld32(tS + c * 32, reinterpret_cast<uint32_t*>(sv) + c * 32);
       tc::wait_ld();
       const int t0 = j * kTcKeys;
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (t0 + kTcKeys - 1 > limit) {              // diagonal / tail tile: mask
+        const int lim = limit - t0;
 #pragma unroll
-        for (int i = 0; i < kTcKeys; ++i) {
-          sv[i] = (t0 + i <= limit) ? sv[i] : -INFINITY;
-          mx4[i & 3] = fmaxf(mx4[i & 3], sv[i]);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < kTcKeys; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], sv[i]);
+        for (int i = 0; i < kTcKeys; ++i) sv[i] = i <= lim ? sv[i] : -INFINITY;
       }
-      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;  // scale > 0
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int i = 0; i < kTcKeys; i += 8) {
+        mx4[0] = max3f(mx4[0], sv[i + 0], sv[i + 1]);
+        mx4[1] = max3f(mx4[1], sv[i + 2], sv[i + 3]);
+        mx4[2] = max3f(mx4[2], sv[i + 4], sv[i + 5]);
+        mx4[3] = max3f(mx4[3], sv[i + 6], sv[i + 7]);
+      }
+      const float mx = max3f(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * sl2;  // scale > 0
       float alpha = 1.f;
       bool resc = false;
       if (m_ref == -INFINITY) {
@@ -339,16 +406,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         l *= alpha;
       }
       const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
-      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint64_t sc2 = f32x2(sl2, sl2), nm2 = f32x2(neg_m, neg_m);
+      uint64_t rs2[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
       uint32_t pk[kTcKeys / 2];
 #pragma unroll
       for (int i = 0; i < kTcKeys; i += 2) {
-        const float e0 = fast_exp2(fmaf(sv[i], sl2, neg_m));
-        const float e1 = fast_exp2(fmaf(sv[i + 1], sl2, neg_m));
-        rs4[(i >> 1) & 3] += e0 + e1;
+        float x0, x1;
+        f32x2_split(ffma2(f32x2(sv[i], sv[i + 1]), sc2, nm2), x0, x1);
+        // PA_EXP_POLY_OF_8 pairs in eight on the FMA pipe, the rest on MUFU
+        const bool poly = ((i >> 1) & 7) >= 8 - PA_EXP_POLY_OF_8;
+        const float e0 = poly ? exp2_poly(x0) : fast_exp2(x0);
+        const float e1 = poly ? exp2_poly(x1) : fast_exp2(x1);
+        rs2[(i >> 1) & 1] = fadd2(rs2[(i >> 1) & 1], f32x2(e0, e1));
         pk[i >> 1] = pack_bf16(e0, e1);
       }
-      l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+      {
+        float a0, a1, b0, b1;
+        f32x2_split(rs2[0], a0, a1);
+        f32x2_split(rs2[1], b0, b1);
+        l += (a0 + a1) + (b0 + b1);
+      }
       tc::st32(tS, pk);                            // P over the first 64 S columns
       tc::st32(tS + 32, pk + 32);
       if (__any_sync(0xffffffffu, resc)) {
