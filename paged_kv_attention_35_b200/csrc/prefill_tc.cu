@@ -121,6 +121,27 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   return d;
 }
 
+// Two exponentials per MUFU instruction: 2^x for a pair of fp32 arguments via
+// ex2.approx.f16x2.  The arguments are <= 8 (lazy rescale) and the results are
+// rounded to bf16 for P right after; the f16 argument's half-ulp error (at most
+// 2^-8 absolute for |x| < 16, i.e. 0.27% relative on p) is of the order of
+// that bf16 rounding, and x < -16 only reaches weights below 2^-16.
+// Off by default: the extra conversions cost more issue slots than the MUFU
+// time they save in this kernel (measured 454 vs 509 TFLOP/s on the
+// prefix-cached prefill workload); likewise the polynomial share below.
+#ifndef PA_EXP_F16X2
+#define PA_EXP_F16X2 0
+#endif
+__device__ __forceinline__ void exp2_pair_f16(float x0, float x1, float& e0, float& e1) {
+  uint32_t h, e;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(x1), "f"(x0));
+  asm("ex2.approx.f16x2 %0, %1;" : "=r"(e) : "r"(h));
+  asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "cvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
+      : "=f"(e0), "=f"(e1)
+      : "r"(e));
+}
+
 constexpr int kBtCache = 256;    // block-table entries staged in shared memory
 #ifndef PA_EXP_POLY_OF_8
 #define PA_EXP_POLY_OF_8 0         // exponential pairs out of every 8 computed by exp2_poly
@@ -326,30 +347,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int j = 0; ok && j < n; ++j) {
         const int iv = 2 * j + 1, vslot = iv % kRing;
         const bool vz = zero_tail && j == n - 1;
-        bool v_ready = false, k_next = false;
-        for (int t = 0; t < 2 && ok; ++t) {
+        // operands first (normally resident long before the softmax is done), so
+        // nothing but the P handshake sits between consecutive MMA groups
+        if (!tc_wait(vz ? &bar->vz_ready : &bar->kv_full[vslot], vz ? 0u : (uint32_t)((iv / kRing) & 1),
+                     abort_flag, p.err_flag) ||
+            (j + 1 < n && !wait_k(j + 1))) {
+          ok = false;
+          break;
+        }
+        for (int t = 0; t < 2; ++t) {
           if (j >= ntile[t]) continue;
           if (!tc_wait(&bar->p_full[t], j & 1, abort_flag, p.err_flag)) { ok = false; break; }
-          if (!v_ready) {
-            if (!tc_wait(vz ? &bar->vz_ready : &bar->kv_full[vslot], vz ? 0u : (uint32_t)((iv / kRing) & 1),
-                         abort_flag, p.err_flag)) { ok = false; break; }
-            v_ready = true;
-          }
           tc::fence_after_sync();
           const uint32_t aV = smem_u32(sKV + vslot * kTile);
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
             tc::mma_ts(tmem + 256 * t + 128, tmem + 256 * t + ks * 8,
                        tc::sdesc_sw128(aV + ks * 2048, kHalf, 1024), idO, (j > 0 || ks > 0));
-          tc::commit(&bar->pv_done[t]);
-          if (j + 1 < ntile[t]) {
-            if (!k_next) {
-              if (!wait_k(j + 1)) { ok = false; break; }
-              k_next = true;
-              tc::fence_after_sync();
-            }
-            issue_s(t, j + 1);
-          }
+          if (j == ntile[t] - 1) tc::commit(&bar->pv_done[t]);   // the epilogue waits on it
+          if (j + 1 < ntile[t]) issue_s(t, j + 1);
         }
         if (!ok) break;
         tc::commit(&bar->kv_empty[vslot]);                 // V_j consumed
@@ -415,8 +431,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         f32x2_split(ffma2(f32x2(sv[i], sv[i + 1]), sc2, nm2), x0, x1);
         // PA_EXP_POLY_OF_8 pairs in eight on the FMA pipe, the rest on MUFU
         const bool poly = ((i >> 1) & 7) >= 8 - PA_EXP_POLY_OF_8;
-        const float e0 = poly ? exp2_poly(x0) : fast_exp2(x0);
-        const float e1 = poly ? exp2_poly(x1) : fast_exp2(x1);
+        float e0, e1;
+        if (poly) {
+          e0 = exp2_poly(x0);
+          e1 = exp2_poly(x1);
+        } else if (PA_EXP_F16X2) {
+          exp2_pair_f16(x0, x1, e0, e1);
+        } else {
+          e0 = fast_exp2(x0);
+          e1 = fast_exp2(x1);
+        }
         rs2[(i >> 1) & 1] = fadd2(rs2[(i >> 1) & 1], f32x2(e0, e1));
         pk[i >> 1] = pack_bf16(e0, e1);
       }
@@ -445,7 +469,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lane == 0) mbar_arrive(&bar->p_full[t]);
     }
     // epilogue: O / l -> bf16
-    if (nt > 0 && ok && tc_wait(&bar->pv_done[t], (nt - 1) & 1, abort_flag, p.err_flag)) {
+    if (nt > 0 && ok && tc_wait(&bar->pv_done[t], 0, abort_flag, p.err_flag)) {
       tc::fence_after_sync();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const bool store = q0 + r < q_len;
