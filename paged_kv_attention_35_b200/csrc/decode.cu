@@ -97,6 +97,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   uint64_t* empty = full + STAGES;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + STAGES);
 
+  pdl_wait();
+  pdl_trigger();
   const int split = blockIdx.x;
   const int kvh = blockIdx.y / p.qtiles;
   const int qt = blockIdx.y % p.qtiles;
@@ -358,6 +360,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 // out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
 template <int D>
 __global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeParams p) {
+  pdl_wait();
+  pdl_trigger();
   const int h = blockIdx.x, seq = blockIdx.y, d = threadIdx.x;
   const int L = clamp_len(__ldg(p.context_lens + seq), p);
   const int n = (L + p.partition - 1) / p.partition;
@@ -388,12 +392,11 @@ static pa_status launch_decode_d(const DecodeArgs& a, const CUtensorMap& mk, con
     attr_done = true;
   }
   dim3 grid(a.max_splits, a.hkv * prm.qtiles, a.num_seqs);
-  decode_kernel<D, kDecStages><<<grid, kDecThreads, smem, a.stream>>>(mk, mv, prm);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(decode_kernel<D, kDecStages>, grid, dim3(kDecThreads), smem, a.stream,
+                             mk, mv, prm);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   if (a.max_splits > 1) {
-    decode_reduce_kernel<D><<<dim3(a.hq, a.num_seqs), D, 0, a.stream>>>(prm);
-    e = cudaGetLastError();
+    e = launch_pdl(decode_reduce_kernel<D>, dim3(a.hq, a.num_seqs), dim3(D), 0, a.stream, prm);
     if (e != cudaSuccess) return cuda_fail(e, "decode reduce launch");
   }
   return PA_OK;

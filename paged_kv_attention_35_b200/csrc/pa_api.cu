@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -19,6 +20,14 @@ namespace pa {
 __device__ unsigned int g_watchdog = 0;
 
 static thread_local std::string t_last_error;
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("PA_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
 
 pa_status fail(pa_status s, const std::string& msg) {
   t_last_error = msg;

@@ -123,6 +123,17 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ----------------------------------------------- programmatic dependent launch
+// Kernels are launched with programmatic stream serialization: a kernel may be
+// scheduled while the previous kernel on the stream is still running, and
+// waits here before reading any input (the wait returns once that kernel has
+// completed and its writes are visible; without the launch attribute it
+// returns at once).  The trigger lets the next kernel be scheduled early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // --------------------------------------------------------- named barriers
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

@@ -8,10 +8,30 @@
 #include <stdint.h>
 
 #include <string>
+#include <utility>
 
 #include "../../include/pagedattn.h"
 
 namespace pa {
+
+// Launches `kern` on `stream` with programmatic stream serialization allowed
+// (the kernels call pdl_wait() before reading inputs), unless PA_PDL=0.
+bool pdl_enabled();
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Records `msg` as this thread's last error and returns `s`.
 pa_status fail(pa_status s, const std::string& msg);

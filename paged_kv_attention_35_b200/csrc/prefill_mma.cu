@@ -97,6 +97,8 @@ __global__ void __launch_bounds__(kPfThreads, 2)
   uint64_t* ready = empty + STAGES;                // last tile zeroed (see below)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ready + 1);
 
+  pdl_wait();
+  pdl_trigger();
   const int qtile = blockIdx.x;
   const int h = blockIdx.y;
   const int seq = blockIdx.z;
@@ -329,8 +331,8 @@ static pa_status launch_prefill_mma_d(const PrefillArgs& a, const CUtensorMap& m
     attr_done = true;
   }
   dim3 grid((a.max_seqlen_q + kPfTile - 1) / kPfTile, a.hq, a.num_seqs);
-  prefill_mma_kernel<D, kPfStages><<<grid, kPfThreads, smem, a.stream>>>(mk, mv, prm);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(prefill_mma_kernel<D, kPfStages>, grid, dim3(kPfThreads), smem,
+                             a.stream, mk, mv, prm);
   if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
   return PA_OK;
 }

@@ -181,6 +181,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // pair 0 = the sequence's last two query tiles (they see the most keys), so
   // launch order is longest first and every CTA but possibly a sequence's
   // first carries two tiles; tile A is the later one of the pair.
+  pdl_wait();
+  pdl_trigger();
   const int pp = blockIdx.x;
   const int h = blockIdx.y, seq = blockIdx.z;
   const int kvh = h / p.group;
@@ -540,8 +542,8 @@ pa_status launch_prefill_tc(const PrefillArgs& a) {
   }
   if (a.hq > 65535) return fail(PA_ERR_UNSUPPORTED, "too many heads");
   dim3 grid((a.max_seqlen_q + 2 * kTcRows - 1) / (2 * kTcRows), a.hq, a.num_seqs);
-  prefill_tc_kernel<<<grid, kTcThreads, smem, a.stream>>>(mq, mk, mv, prm);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(prefill_tc_kernel, grid, dim3(kTcThreads), smem, a.stream, mq, mk, mv,
+                             prm);
   if (e != cudaSuccess) return cuda_fail(e, "prefill_tc launch");
   return PA_OK;
 }

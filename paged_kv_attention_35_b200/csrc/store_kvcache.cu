@@ -29,6 +29,8 @@ __global__ void __launch_bounds__(256) store_kvcache_kernel(
     int64_t value_stride16, uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
     const int32_t* __restrict__ slots, int num_tokens, int row16, int rows_per_cta,
     int64_t num_slots, int32_t* err_flag) {
+  pdl_wait();
+  pdl_trigger();
   // thread -> (row within the CTA, first chunk); long rows are strided by the CTA
   const bool long_row = row16 >= (int)blockDim.x;
   const int lr = long_row ? 0 : (int)threadIdx.x / row16;
@@ -61,11 +63,11 @@ pa_status launch_store(const void* key, const void* value, int64_t key_stride,
   int rows_per_cta = row16 >= threads ? 1 : threads / row16;
   int64_t grid = (num_tokens + rows_per_cta - 1) / rows_per_cta;
   if (grid > INT32_MAX) return fail(PA_ERR_UNSUPPORTED, "too many tokens");
-  store_kvcache_kernel<<<(unsigned)grid, threads, 0, stream>>>(
-      static_cast<const uint4*>(key), static_cast<const uint4*>(value), key_stride / 8,
-      value_stride / 8, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), slots,
-      num_tokens, row16, rows_per_cta, num_slots, err_flag);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(store_kvcache_kernel, dim3((unsigned)grid), dim3(threads), 0, stream,
+                             static_cast<const uint4*>(key), static_cast<const uint4*>(value),
+                             key_stride / 8, value_stride / 8, static_cast<uint4*>(k_cache),
+                             static_cast<uint4*>(v_cache), slots, num_tokens, row16, rows_per_cta,
+                             num_slots, err_flag);
   if (e != cudaSuccess) return cuda_fail(e, "store_kvcache launch");
   return PA_OK;
 }
