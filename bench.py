@@ -8,8 +8,8 @@ sequence's new K/V row into the pool + paged decode attention over the batch.
 
 Metric: decode-step KV GB/s (algorithmic bytes of the step / step time), with
 tokens/s (sequences decoded per second for this layer) beside it.  Inputs are
-resident in HBM when timing starts; L2 is flushed (a 512 MiB write) before
-every timed step and each step is bracketed by CUDA events on the launching
+resident in HBM when timing starts; L2 is flushed (a 512 MiB write, then a
+512 MiB read so the write's dirty lines are gone too) before every timed step and each step is bracketed by CUDA events on the launching
 stream.  With --gpus N (torchrun, one rank per GPU) every rank runs its own
 replica of the workload (no collective on the data path: "scaling": "weak")
 and the time is the max over ranks.
@@ -108,26 +108,41 @@ class ClockSampler:
 
 # --------------------------------------------------------------------- timing
 class Timer:
-    """Per-step CUDA-event timing on the current stream, L2 flushed before each step."""
+    """Per-step CUDA-event timing on the current stream, L2 flushed before each step.
+
+    The flush writes a 512 MiB buffer (4x the 126 MB L2) and then reads another
+    512 MiB buffer: the write evicts every line, the read pushes the write's own
+    dirty lines back to HBM before the step starts, so the timed kernels neither
+    find their inputs in L2 nor pay for write-backs that are not theirs."""
 
     def __init__(self, torch, flush_bytes=512 << 20):
         self.torch = torch
         self.flush_buf = torch.empty(flush_bytes, dtype=torch.uint8, device="cuda")
+        self.read_buf = torch.zeros(flush_bytes // 4, dtype=torch.float32, device="cuda")
 
     def flush(self):
         self.flush_buf.fill_(1)
+        self.read_buf.sum()
 
     def time_steps(self, fn, steps, marks=1):
         """Runs `fn(ev)` `steps` times; fn records its own events in `ev` (list of marks+1 events).
-        Returns per-step lists of segment durations in ms."""
+        Returns per-step lists of segment durations in ms.  Python's garbage collector
+        is paused meanwhile so a collection cannot stall the launches of a step."""
+        import gc
         torch = self.torch
         segs = []
-        for _ in range(steps):
-            self.flush()
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(marks + 1)]
-            fn(ev)
-            segs.append(ev)
-        torch.cuda.synchronize()
+        gc_was = gc.isenabled()
+        gc.disable()
+        try:
+            for _ in range(steps):
+                self.flush()
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(marks + 1)]
+                fn(ev)
+                segs.append(ev)
+            torch.cuda.synchronize()
+        finally:
+            if gc_was:
+                gc.enable()
         return [[e[i].elapsed_time(e[i + 1]) for i in range(marks)] for e in segs]
 
 
@@ -167,6 +182,9 @@ def bench_decode(torch, w, steps, warmup, timer, dist=None, world=1, partition=0
     between them), then `steps` decode launches alone (the roofline's kernel)."""
     from paged_kv_attention_35_b200 import ops
     stream = torch.cuda.current_stream()
+    need = ops.decode_workspace_size(w.B, w.hq, w.hkv, w.d, w.max_context_len, partition)
+    if need > w.d_ws.numel():
+        w.d_ws = torch.empty(need, dtype=torch.uint8, device="cuda")
     for _ in range(warmup):
         w.step(partition_size=partition)
     barrier(torch, dist, world)
@@ -317,7 +335,7 @@ def ours(args):
             "config": {"workload": spec.name, "num_seqs": w.B, "context_lens": "U[128,4096]",
                        "sum_context": int(sum(w.lens)), "num_q_heads": w.hq, "num_kv_heads": w.hkv,
                        "head_dim": w.d, "block_size": w.bs, "num_blocks": w.nb,
-                       "partition": args.partition or "auto", "l2": "flushed (512 MiB write) before every step",
+                       "partition": args.partition or "auto", "l2": "flushed before every step (512 MiB write, then 512 MiB read)",
                        "parallelism": f"replicas x{world}"},
             "tokens_per_s": round(tokens_s, 1),
             "breakdown_ms": {"decode_alone": round(r["decode_ms"], 4),
