@@ -85,12 +85,15 @@ def prepare_prefill(seqs, block_size: int) -> PrefillMetadata:
 
 
 def prepare_decode(seqs, block_size: int) -> DecodeMetadata:
-    slots = np.empty(len(seqs), dtype=np.int32)
-    lens = np.empty(len(seqs), dtype=np.int32)
+    slots = [0] * len(seqs)
+    lens = [0] * len(seqs)
     for i, s in enumerate(seqs):
         n = len(s)
-        slots[i] = slots_for(s.block_table, n - 1, n, block_size)[0]
+        pos = n - 1                      # the newest token
+        slots[i] = s.block_table[pos // block_size] * block_size + pos % block_size
         lens[i] = n
+    slots = np.asarray(slots, dtype=np.int32)
+    lens = np.asarray(lens, dtype=np.int32)
     return DecodeMetadata(slot_mapping=slots, context_lens=lens,
                           block_tables=block_tables_array(seqs),
                           max_context_len=int(lens.max()) if len(seqs) else 0)
