@@ -210,24 +210,42 @@ def bench_decode(torch, w, steps, warmup, timer, dist=None, world=1, partition=0
 
 
 def bench_decode_e2e(torch, w, steps, warmup, timer):
-    """Same step through host buffers: H2D of the step's inputs, kernels, D2H of the output."""
+    """Same step through host buffers: H2D of the step's inputs, kernels, D2H of the output.
+
+    The step's inputs (q, new K/V rows, slot_mapping, block tables, context lengths)
+    sit in one pinned staging buffer at 256-byte aligned offsets and go up in one
+    copy per step into one device buffer whose views the calls take, as an
+    engine would stage a step (one DMA instead of six fixed-cost transfers)."""
     from paged_kv_attention_35_b200 import ops
     stream = torch.cuda.current_stream()
-    h = {
-        "q": w.q.pin_memory(), "k": w.new_k.pin_memory(), "v": w.new_v.pin_memory(),
-        "slots": torch.from_numpy(w.decode_slots).pin_memory(),
-        "bt": torch.from_numpy(w.block_tables).pin_memory(),
-        "cl": torch.tensor(w.lens, dtype=torch.int32).pin_memory(),
+    src = {
+        "q": w.q, "k": w.new_k, "v": w.new_v,
+        "slots": torch.from_numpy(w.decode_slots),
+        "bt": torch.from_numpy(w.block_tables),
+        "cl": torch.tensor(w.lens, dtype=torch.int32),
     }
+    offs, total = {}, 0
+    for k, t in src.items():
+        offs[k] = total
+        total += (t.numel() * t.element_size() + 255) // 256 * 256
+    h_buf = torch.empty(total, dtype=torch.uint8).pin_memory()
+    d_buf = torch.empty(total, dtype=torch.uint8, device="cuda")
+
+    def view(buf, k):
+        t = src[k]
+        n = t.numel() * t.element_size()
+        return buf[offs[k]:offs[k] + n].view(t.dtype).view(t.shape)
+
+    for k, t in src.items():
+        view(h_buf, k).copy_(t.contiguous())
+    d = {k: view(d_buf, k) for k in src}
     out_h = torch.empty(w.d_out.shape, dtype=torch.bfloat16).pin_memory()
-    d = {"q": w.d_q, "k": w.d_new_k, "v": w.d_new_v, "slots": w.d_slots, "bt": w.d_bt, "cl": w.d_cl}
-    h2d = sum(t.numel() * t.element_size() for t in h.values())
+    h2d = total
     d2h = out_h.numel() * out_h.element_size()
 
     def one(ev):
         ev[0].record(stream)
-        for k in h:
-            d[k].copy_(h[k], non_blocking=True)
+        d_buf.copy_(h_buf, non_blocking=True)
         ops.store_kvcache(d["k"], d["v"], w.kc, w.vc, d["slots"])
         ops.decode(d["q"], w.kc, w.vc, d["bt"], d["cl"], w.max_context_len, out=w.d_out,
                    workspace=w.d_ws)
@@ -395,7 +413,10 @@ def secondary(torch, args, timer, pk):
     if not args.no_replay:
         try:
             from paged_kv_attention_35_b200.replay import run_replay_bench
-            out["trace_replay"] = run_replay_bench(torch, max_steps=args.replay_steps)
+            out["trace_replay"] = run_replay_bench(torch, max_steps=args.replay_steps, graphs=False)
+            g = run_replay_bench(torch, max_steps=args.replay_steps, graphs=True)
+            out["trace_replay_graphs"] = {k: g[k] for k in (
+                "tokens_per_s", "wall_s", "steps", "graph_steps", "graph_captures", "decode_kv_GBs")}
         except ImportError:
             pass
     return out
@@ -425,7 +446,7 @@ def only(args):
                "GBs": round(nbytes / (ms * 1e-3) / 1e9, 1)}
     else:
         from paged_kv_attention_35_b200.replay import run_replay_bench
-        res = run_replay_bench(torch, max_steps=args.replay_steps)
+        res = run_replay_bench(torch, max_steps=args.replay_steps, graphs=args.graphs)
     print(json.dumps(res), flush=True)
 
 
@@ -553,6 +574,7 @@ def main():
     ap.add_argument("--no-replay", action="store_true")
     ap.add_argument("--replay-steps", type=int, default=0)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--graphs", action="store_true", help="--only replay: graph-replayed decode steps")
     ap.add_argument("--only", choices=["prefill", "decode_gqa", "store", "replay"], default=None,
                     help="time one secondary workload alone (for profiling) and print its JSON")
     args = ap.parse_args()

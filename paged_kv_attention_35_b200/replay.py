@@ -15,6 +15,15 @@ then ``prefill_varlen`` or ``decode`` into a scratch output -> postprocess
 (append tokens, finish, free).  All launches go to the current stream; the
 host runs ahead of the GPU except where it reuses a pinned staging buffer.
 
+With ``graphs=True`` a decode step's 28 layers run as one captured CUDA graph
+("CUDA Graphs", lnwmold.com item: decode is captured for common batch sizes
+to cut launch overhead).  A graph is keyed by the batch size rounded up to a
+multiple of 16, the longest context rounded up to 512 and the ring offset of
+the step; the metadata goes to fixed device buffers the graph reads (padding
+rows: slot -1, context length 0, which the kernels skip / answer with zeros).
+On the first step of a key the layers run eagerly and the graph is captured
+for the next ones.  Prefill steps always run eagerly.
+
 ``slot_writer`` records, for every pool slot, which (step, packed row) last
 wrote it -- the same for every layer, since all layers share the block tables.
 With the CPU copy of the ring this lets a checker rebuild exactly what any
@@ -24,6 +33,7 @@ sequence's K/V history holds on the GPU.
 from __future__ import annotations
 
 import time
+from collections import OrderedDict
 from dataclasses import dataclass
 
 import numpy as np
@@ -54,7 +64,8 @@ class ReplayConfig:
 
 
 class Replay:
-    def __init__(self, cfg: ReplayConfig, device="cuda", record=False):
+    def __init__(self, cfg: ReplayConfig, device="cuda", record=False, graphs=False,
+                 max_graphs=64):
         from . import ops
         self.ops = ops
         self.cfg = cfg
@@ -97,9 +108,24 @@ class Replay:
         self.d_meta = torch.empty(self.meta_len, dtype=torch.int32, device=device)
         self.ws = torch.empty(1 << 20, dtype=torch.uint8, device=device)
         self.slot_writer = np.full((c.num_blocks * c.block_size, 2), -1, dtype=np.int64)
+        self.graphs = graphs
+        if graphs:
+            # fixed metadata buffers of graph-replayed decode steps: slots [S],
+            # context_lens [S], block_tables [S, width] (S = max_num_seqs)
+            S = c.max_num_seqs
+            self.g_width = width
+            self.g_meta = torch.empty(2 * S + S * width, dtype=torch.int32, device=device)
+            self.g_pinned = [torch.empty(self.g_meta.numel(), dtype=torch.int32).pin_memory()
+                             for _ in range(2)]
+            self.g_pinned_ev = [None, None]
+            self.graph_cache = OrderedDict()
+            self.max_graphs = max_graphs
+            need = ops.decode_workspace_size(S, hq, hkv, d, self._ctx_bucket(c.max_model_len))
+            self.g_ws = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
         self.step_idx = 0
         self.stats = dict(steps=0, prefill_steps=0, decode_steps=0, prefill_tokens=0,
-                          decode_tokens=0, decode_kv_bytes=0, launches=0)
+                          decode_tokens=0, decode_kv_bytes=0, launches=0, graph_steps=0,
+                          graph_captures=0)
         self.samples = {}          # (step, layer) -> captured output and the step's metadata
         self.sample_at = set()     # (step, layer) pairs to capture (needs record=True)
         self.snap = {}             # step -> slot_writer after that step's stores
@@ -126,6 +152,67 @@ class Replay:
         ev.record()
         self.pinned_ev[b] = ev
         return [self.d_meta[o:o + int(np.prod(sh))].view(*sh) for o, sh in views]
+
+    # ----------------------------------------------------------- graph steps
+    def _batch_bucket(self, n: int) -> int:
+        return min(-(-n // 16) * 16, self.cfg.max_num_seqs)
+
+    def _ctx_bucket(self, L: int) -> int:
+        return min(-(-L // 512) * 512, self.cfg.max_model_len)
+
+    def _graph_views(self, nb: int):
+        S, w = self.cfg.max_num_seqs, self.g_width
+        m = self.g_meta
+        return m[:nb], m[S:S + nb], m[2 * S:2 * S + nb * w].view(nb, w)
+
+    def _decode_layers(self, nb: int, lb: int, step: int, slots, cl, bt, out):
+        c, ops = self.cfg, self.ops
+        for layer in range(c.num_layers):
+            r = self.ring_index(step, layer)
+            kc, vc = self.k_pools[layer], self.v_pools[layer]
+            ops.store_kvcache(self.k_ring[r, :nb], self.v_ring[r, :nb], kc, vc, slots)
+            ops.decode(self.q_ring[r, :nb], kc, vc, bt, cl, lb, out=out, workspace=self.g_ws)
+
+    def _decode_graph_step(self, md, n: int):
+        """One decode step through a captured graph (see the module docstring)."""
+        c = self.cfg
+        S, w = c.max_num_seqs, self.g_width
+        nb, lb = self._batch_bucket(n), self._ctx_bucket(md.max_context_len)
+        b = self.step_idx & 1
+        if self.g_pinned_ev[b] is not None:
+            self.g_pinned_ev[b].synchronize()
+        host = self.g_pinned[b].numpy()
+        host[:nb] = -1
+        host[:n] = md.slot_mapping
+        host[S:S + nb] = 0
+        host[S:S + n] = md.context_lens
+        btv = host[2 * S:2 * S + nb * w].reshape(nb, w)
+        btv[:] = -1
+        btv[:n, :md.block_tables.shape[1]] = md.block_tables
+        used = 2 * S + nb * w
+        self.g_meta[:used].copy_(self.g_pinned[b][:used], non_blocking=True)
+        ev = torch.cuda.Event()
+        ev.record()
+        self.g_pinned_ev[b] = ev
+        slots, cl, bt = self._graph_views(nb)
+        out = self.out[:nb]
+        key = (nb, lb, (self.step_idx * c.num_layers) % c.ring)
+        g = self.graph_cache.get(key)
+        if g is None:
+            # this step eagerly (also the lazy set-up of every launch), then the capture
+            self._decode_layers(nb, lb, self.step_idx, slots, cl, bt, out)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self._decode_layers(nb, lb, self.step_idx, slots, cl, bt, out)
+            self.graph_cache[key] = g
+            self.stats["graph_captures"] += 1
+            if len(self.graph_cache) > self.max_graphs:
+                self.graph_cache.popitem(last=False)
+        else:
+            self.graph_cache.move_to_end(key)
+            g.replay()
+            self.stats["graph_steps"] += 1
+        return out[:n]
 
     # -------------------------------------------------------------------- step
     def step(self) -> bool:
@@ -155,7 +242,15 @@ class Replay:
                 c.head_dim * 4 * c.num_layers
         out = self.out[:n]
         captured = False
-        for layer in range(c.num_layers):
+        if self.graphs and not is_prefill:
+            out = self._decode_graph_step(md, n)
+            last = c.num_layers - 1
+            if self.record == "all" or (self.step_idx, last) in self.sample_at:
+                self.samples[(self.step_idx, last)] = dict(
+                    is_prefill=False, md=md, out=out.cpu().clone(),
+                    block_tables=[list(s.block_table) for s in seqs], lens=[len(s) for s in seqs])
+                captured = True
+        for layer in range(0 if (self.graphs and not is_prefill) else c.num_layers):
             r = self.ring_index(self.step_idx, layer)
             kc, vc = self.k_pools[layer], self.v_pools[layer]
             ops.store_kvcache(self.k_ring[r, :n], self.v_ring[r, :n], kc, vc, slots)
@@ -170,9 +265,13 @@ class Replay:
                     is_prefill=is_prefill, md=md, out=out.cpu().clone(),
                     block_tables=[list(s.block_table) for s in seqs], lens=[len(s) for s in seqs])
                 captured = True
-        self.stats["launches"] += c.num_layers * (2 if is_prefill else (
-            3 if ops.decode_workspace_size(n, c.num_q_heads, c.num_kv_heads, c.head_dim,
-                                           md.max_context_len) > 0 else 2))
+        if self.graphs and not is_prefill:
+            nb, lb = self._batch_bucket(n), self._ctx_bucket(md.max_context_len)
+            split = ops.decode_workspace_size(nb, c.num_q_heads, c.num_kv_heads, c.head_dim, lb) > 0
+        else:
+            split = not is_prefill and ops.decode_workspace_size(
+                n, c.num_q_heads, c.num_kv_heads, c.head_dim, md.max_context_len) > 0
+        self.stats["launches"] += c.num_layers * (3 if split else 2)
         if self.record:
             sm = md.slot_mapping.astype(np.int64)
             self.slot_writer[sm, 0] = self.step_idx
@@ -205,10 +304,10 @@ class Replay:
         return st
 
 
-def run_replay_bench(torch_mod=None, max_steps=0, cfg: ReplayConfig | None = None):
+def run_replay_bench(torch_mod=None, max_steps=0, cfg: ReplayConfig | None = None, graphs=True):
     """The trace replay as a bench workload: tokens/s over the whole loop."""
     cfg = cfg or ReplayConfig()
-    rp = Replay(cfg)
+    rp = Replay(cfg, graphs=graphs)
     torch.cuda.synchronize()
     st = rp.run(max_steps=max_steps)
     tokens = st["prefill_tokens"] + st["decode_tokens"]
@@ -219,6 +318,7 @@ def run_replay_bench(torch_mod=None, max_steps=0, cfg: ReplayConfig | None = Non
         "prefill_tokens": st["prefill_tokens"], "decode_tokens": st["decode_tokens"],
         "preemptions": st["preemptions"], "prefix_hit_tokens": st["prefix_hit_tokens"],
         "finished": st["finished"], "requests": cfg.num_requests, "launches": st["launches"],
+        "graphs": graphs, "graph_steps": st["graph_steps"], "graph_captures": st["graph_captures"],
         "decode_kv_GBs": round(st["decode_kv_bytes"] / st["wall_s"] / 1e9, 1),
         "config": {"layers": cfg.num_layers, "heads": f"{cfg.num_q_heads}/{cfg.num_kv_heads}",
                    "head_dim": cfg.head_dim, "block_size": cfg.block_size,

@@ -92,6 +92,41 @@ def test_small_trace_every_step(cuda_device):
     assert rp.sched.block_manager.num_free_blocks == cfg.num_blocks
 
 
+def _small_cfg():
+    return ReplayConfig(num_requests=14, prompt_lo=5, prompt_hi=70, output_lo=3, output_hi=40,
+                        max_num_seqs=6, max_num_batched_tokens=160, block_size=16, num_blocks=14,
+                        num_layers=2, num_q_heads=8, num_kv_heads=2, head_dim=128, ring=3, seed=4242,
+                        max_model_len=128)
+
+
+def test_small_trace_graphs_every_step(cuda_device):
+    """Decode steps replayed as captured CUDA graphs (padded batch, fixed metadata
+    buffers): every prefill layer and every decode step's last layer against the oracle."""
+    cfg = _small_cfg()
+    rp = Replay(cfg, record="all", graphs=True)
+    st = rp.run()
+    assert st["finished"] == cfg.num_requests
+    assert st["graph_captures"] > 0 and st["graph_steps"] > st["graph_captures"]
+    decode_samples = [k for k in rp.samples if not rp.samples[k]["is_prefill"]]
+    assert decode_samples and all(l == cfg.num_layers - 1 for _, l in decode_samples)
+    for (step, layer) in sorted(rp.samples):
+        check_sample(rp, step, layer)
+    assert rp.sched.block_manager.num_free_blocks == cfg.num_blocks
+
+
+def test_graph_replay_pools_equal_eager(cuda_device):
+    """The same trace eager and graph-replayed leaves bit-identical K/V pools."""
+    cfg = _small_cfg()
+    a = Replay(cfg)
+    a.run()
+    b = Replay(cfg, graphs=True)
+    b.run()
+    torch.cuda.synchronize()
+    for la in range(cfg.num_layers):
+        assert torch.equal(a.k_pools[la].view(torch.int16), b.k_pools[la].view(torch.int16))
+        assert torch.equal(a.v_pools[la].view(torch.int16), b.v_pools[la].view(torch.int16))
+
+
 def test_full_trace_sampled(cuda_device):
     """512 requests, prompt/output U[100,1024], 256 seqs, block 256, 768 blocks, 28 layers."""
     cfg = ReplayConfig()
@@ -105,3 +140,19 @@ def test_full_trace_sampled(cuda_device):
         check_sample(rp, *key, max_seqs=6)
         checked += 1
     assert checked >= 6
+
+
+def test_full_trace_graphs_sampled(cuda_device):
+    """The bench's trace with graph-replayed decode steps, last layer sampled."""
+    cfg = ReplayConfig()
+    rp = Replay(cfg, record=True, graphs=True)
+    last = cfg.num_layers - 1
+    rp.sample_at = {(s, last) for s in (3, 40, 400, 1100, 1900)}
+    st = rp.run()
+    assert st["finished"] == cfg.num_requests
+    assert st["graph_steps"] > 10 * st["graph_captures"]
+    checked = 0
+    for key in sorted(rp.samples):
+        check_sample(rp, *key, max_seqs=6)
+        checked += 1
+    assert checked >= 4
