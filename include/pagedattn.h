@@ -68,6 +68,8 @@ typedef enum { PA_BF16 = 0 } pa_dtype;
 #define PA_FLAG_BLOCK_OOB  2  /* block table entry outside [0, num_blocks)            */
 #define PA_FLAG_LEN_OOB    4  /* context/sequence length outside its declared bounds  */
 #define PA_FLAG_TIMEOUT    8  /* a bounded wait gave up                                */
+#define PA_FLAG_SLOT_MISMATCH 16  /* pa_decode_store: slot_mapping[i] is not the slot of
+                                     sequence i's newest position                    */
 
 typedef void* pa_stream_t;
 
@@ -152,6 +154,36 @@ PA_API pa_status pa_decode(void* out, const void* q, int64_t q_token_stride,
                     int32_t block_size, int32_t num_blocks, float scale,
                     int32_t partition_size, void* workspace, size_t workspace_bytes,
                     pa_dtype dtype, int32_t* err_flag, pa_stream_t stream);
+
+/*
+ * pa_decode_store -- one decode step's store_kvcache and decode in one launch.
+ *
+ * Same result as pa_store_kvcache(key, value, key_token_stride,
+ * value_token_stride, k_cache, v_cache, slot_mapping, num_seqs, ...) followed by
+ * pa_decode(...) with the remaining arguments, when slot_mapping[i] is the pool
+ * slot of sequence i's newest position context_lens[i]-1 (the decode-step
+ * invariant: the slot of position p is block_tables[i][p / block_size] *
+ * block_size + p % block_size, "From Sequences to Blocks", lnwmold.com item;
+ * the new token's K/V are written before attention reads them, "Preparation
+ * before computation", same item).  The CTA of each (sequence, KV head) that
+ * reads that position writes the row first, so the store costs no launch and
+ * no extra pass.  key / value: [num_seqs, Hkv, D] bf16 rows (token strides in
+ * elements, multiples of 8, 16-byte aligned).  slot_mapping[i] < 0 skips the
+ * store of row i; >= num_blocks*block_size is skipped with PA_FLAG_SLOT_OOB;
+ * a slot that breaks the invariant sets PA_FLAG_SLOT_MISMATCH (checked mode)
+ * and the result is then unspecified.  Other arguments, errors and the
+ * workspace as pa_decode.
+ */
+PA_API pa_status pa_decode_store(void* out, const void* q, int64_t q_token_stride,
+                          const void* key, const void* value, int64_t key_token_stride,
+                          int64_t value_token_stride, const int32_t* slot_mapping,
+                          void* k_cache, void* v_cache,
+                          const int32_t* block_tables, int32_t max_blocks_per_seq,
+                          const int32_t* context_lens, int32_t num_seqs, int32_t max_context_len,
+                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                          int32_t block_size, int32_t num_blocks, float scale,
+                          int32_t partition_size, void* workspace, size_t workspace_bytes,
+                          pa_dtype dtype, int32_t* err_flag, pa_stream_t stream);
 
 /*
  * pa_decode_noalloc -- pa_decode for callers that cannot allocate device memory.

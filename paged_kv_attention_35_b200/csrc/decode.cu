@@ -25,6 +25,11 @@
 //    kernel stays bound by HBM.
 //  * positions >= context_len in the last tile are masked to -inf and their V
 //    rows zeroed in shared memory before P V (stale pool rows may hold NaN).
+//  * fused store (pa_decode_store): the CTA whose partition holds a
+//    sequence's newest position first writes that token's K and V rows of its
+//    KV head into the pool at slot_mapping[seq] (the store_kvcache of the
+//    step), orders the writes before its TMA reads with a proxy fence, and
+//    then streams as usual -- no other CTA of the launch reads that slot.
 //  * the 4 warps merge (m, l, O) through shared memory; with one partition
 //    the CTA writes bf16 output, otherwise fp32 partials for the reduce kernel.
 
@@ -54,6 +59,14 @@ struct DecodeParams {
   int partition, max_context_len, max_splits;
   float* ws_o;
   float* ws_ml;
+  // fused store: null slots = plain decode
+  const uint4* new_k;
+  const uint4* new_v;
+  int64_t new_k_stride16, new_v_stride16;   // 16-byte units between tokens
+  const int32_t* slots;
+  uint4* kc;
+  uint4* vc;
+  int hkv;
   int32_t* err_flag;
 };
 
@@ -139,6 +152,26 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 
   if (warp == kDecWarps) {
     // ------------------------------------------------------------ producer
+    if (p.slots && t_end == L) {
+      // fused store of the newest token (position L-1) for this KV head
+      const int slot = __ldg(p.slots + seq);
+      const int lb = (L - 1) >> p.log2_bs;
+      const int bid = __ldg(p.block_tables + (int64_t)seq * p.max_blocks + lb);
+      if (slot >= 0 && bid >= 0 && bid < p.num_blocks &&
+          slot != bid * p.block_size + ((L - 1) & (p.block_size - 1)))
+        raise_flag(p.err_flag, PA_FLAG_SLOT_MISMATCH);
+      if (slot >= p.num_slots) raise_flag(p.err_flag, PA_FLAG_SLOT_OOB);
+      if (slot >= 0 && slot < p.num_slots) {
+        constexpr int C = D / 8;                   // 16-byte chunks per head row
+        const int64_t dst = ((int64_t)slot * p.hkv + kvh) * C;
+        const uint4 kx = __ldg(p.new_k + seq * p.new_k_stride16 + kvh * C + (lane & (C - 1)));
+        if (lane < C) p.kc[dst + lane] = kx;
+        const uint4 vx = __ldg(p.new_v + seq * p.new_v_stride16 + kvh * C + (lane & (C - 1)));
+        if (lane < C) p.vc[dst + lane] = vx;
+      }
+      fence_proxy_async_global();                  // the rows above precede this CTA's TMA reads
+    }
+    __syncwarp();
     if (lane == 0) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
@@ -431,6 +464,16 @@ pa_status launch_decode(const DecodeArgs& a) {
   prm.max_splits = a.max_splits;
   prm.ws_o = a.ws_o;
   prm.ws_ml = a.ws_ml;
+  prm.slots = a.slots;
+  if (a.slots) {
+    prm.new_k = static_cast<const uint4*>(a.new_k);
+    prm.new_v = static_cast<const uint4*>(a.new_v);
+    prm.new_k_stride16 = a.new_k_stride / 8;
+    prm.new_v_stride16 = a.new_v_stride / 8;
+    prm.kc = static_cast<uint4*>(const_cast<void*>(a.k_cache));
+    prm.vc = static_cast<uint4*>(const_cast<void*>(a.v_cache));
+  }
+  prm.hkv = a.hkv;
   prm.err_flag = a.err_flag;
   if ((int64_t)a.hkv * prm.qtiles > 65535) return fail(PA_ERR_UNSUPPORTED, "too many heads");
   if (a.d == 128) return launch_decode_d<128>(a, mk, mv, prm);

@@ -224,14 +224,23 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t n
   return ob + mb;
 }
 
-pa_status pa_decode(void* out, const void* q, int64_t q_token_stride, const void* k_cache,
-                    const void* v_cache, const int32_t* block_tables, int32_t max_blocks_per_seq,
-                    const int32_t* context_lens, int32_t num_seqs, int32_t max_context_len,
-                    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
-                    int32_t block_size, int32_t num_blocks, float scale, int32_t partition_size,
-                    void* workspace, size_t workspace_bytes, pa_dtype dtype, int32_t* err_flag,
-                    pa_stream_t stream) {
-  t_last_error.clear();
+namespace {
+struct FusedStore {
+  const void* key;
+  const void* value;
+  int64_t key_stride, value_stride;
+  const int32_t* slots;
+};
+}  // namespace
+
+static pa_status decode_impl(void* out, const void* q, int64_t q_token_stride, const void* k_cache,
+                             const void* v_cache, const int32_t* block_tables,
+                             int32_t max_blocks_per_seq, const int32_t* context_lens,
+                             int32_t num_seqs, int32_t max_context_len, int32_t num_q_heads,
+                             int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                             int32_t num_blocks, float scale, int32_t partition_size,
+                             void* workspace, size_t workspace_bytes, pa_dtype dtype,
+                             int32_t* err_flag, pa_stream_t stream, const FusedStore* st) {
   pa_status s = check_common(k_cache, v_cache, num_q_heads, num_kv_heads, head_dim, block_size,
                              num_blocks, dtype);
   if (s != PA_OK) return s;
@@ -277,7 +286,55 @@ pa_status pa_decode(void* out, const void* q, int64_t q_token_stride, const void
     a.ws_o = static_cast<float*>(workspace);
     a.ws_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + ob);
   }
+  if (st) {
+    a.new_k = st->key;
+    a.new_v = st->value;
+    a.new_k_stride = st->key_stride;
+    a.new_v_stride = st->value_stride;
+    a.slots = st->slots;
+  }
   return launch_decode(a);
+}
+
+pa_status pa_decode(void* out, const void* q, int64_t q_token_stride, const void* k_cache,
+                    const void* v_cache, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                    const int32_t* context_lens, int32_t num_seqs, int32_t max_context_len,
+                    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                    int32_t block_size, int32_t num_blocks, float scale, int32_t partition_size,
+                    void* workspace, size_t workspace_bytes, pa_dtype dtype, int32_t* err_flag,
+                    pa_stream_t stream) {
+  t_last_error.clear();
+  return decode_impl(out, q, q_token_stride, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                     context_lens, num_seqs, max_context_len, num_q_heads, num_kv_heads, head_dim,
+                     block_size, num_blocks, scale, partition_size, workspace, workspace_bytes,
+                     dtype, err_flag, stream, nullptr);
+}
+
+pa_status pa_decode_store(void* out, const void* q, int64_t q_token_stride, const void* key,
+                          const void* value, int64_t key_token_stride, int64_t value_token_stride,
+                          const int32_t* slot_mapping, void* k_cache, void* v_cache,
+                          const int32_t* block_tables, int32_t max_blocks_per_seq,
+                          const int32_t* context_lens, int32_t num_seqs, int32_t max_context_len,
+                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                          int32_t block_size, int32_t num_blocks, float scale,
+                          int32_t partition_size, void* workspace, size_t workspace_bytes,
+                          pa_dtype dtype, int32_t* err_flag, pa_stream_t stream) {
+  t_last_error.clear();
+  if (num_seqs > 0) {
+    if (!key || !value || !slot_mapping) return fail(PA_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned16(key) || !aligned16(value))
+      return fail(PA_ERR_INVALID_ARG, "key/value must be 16-byte aligned");
+    const int64_t row = (int64_t)num_kv_heads * head_dim;
+    if (key_token_stride < row || value_token_stride < row)
+      return fail(PA_ERR_INVALID_ARG, "token stride smaller than num_kv_heads*head_dim");
+    if (key_token_stride % 8 || value_token_stride % 8)
+      return fail(PA_ERR_INVALID_ARG, "token strides must be multiples of 8 elements (16 bytes)");
+  }
+  const FusedStore st{key, value, key_token_stride, value_token_stride, slot_mapping};
+  return decode_impl(out, q, q_token_stride, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                     context_lens, num_seqs, max_context_len, num_q_heads, num_kv_heads, head_dim,
+                     block_size, num_blocks, scale, partition_size, workspace, workspace_bytes,
+                     dtype, err_flag, stream, &st);
 }
 
 pa_status pa_prefill_varlen(void* out, const void* q, int64_t q_token_stride, const void* k_cache,

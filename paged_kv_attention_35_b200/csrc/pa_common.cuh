@@ -123,6 +123,11 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// The same for global memory: generic stores before later TMA reads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // ----------------------------------------------- programmatic dependent launch
 // Kernels are launched with programmatic stream serialization: a kernel may be
 // scheduled while the previous kernel on the stream is still running, and

@@ -60,6 +60,12 @@ struct DecodeArgs {
   int max_splits;      // ceil(max_context_len / partition)
   float* ws_o;         // [B, Hq, max_splits, D]
   float* ws_ml;        // [B, Hq, max_splits, 2]
+  // fused store (pa_decode_store): row i of new_k / new_v goes to pool slot
+  // slots[i] before attention; null slots = plain decode
+  const void* new_k;
+  const void* new_v;
+  int64_t new_k_stride, new_v_stride;   // elements between tokens
+  const int32_t* slots;
   int32_t* err_flag;
   cudaStream_t stream;
 };

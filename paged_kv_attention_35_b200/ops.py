@@ -27,7 +27,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 PA_OK = 0
 PA_BF16 = 0
-FLAG_SLOT_OOB, FLAG_BLOCK_OOB, FLAG_LEN_OOB, FLAG_TIMEOUT = 1, 2, 4, 8
+FLAG_SLOT_OOB, FLAG_BLOCK_OOB, FLAG_LEN_OOB, FLAG_TIMEOUT, FLAG_SLOT_MISMATCH = 1, 2, 4, 8, 16
 STATUS = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_WORKSPACE",
           4: "PA_ERR_CUDA"}
 
@@ -42,6 +42,9 @@ SIGNATURES = {
     "pa_decode_workspace_size": ([_i32, _i32, _i32, _i32, _i32, _i32], _sz),
     "pa_decode": ([_p, _p, _i64, _p, _p, _p, _i32, _p, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
                    _f32, _i32, _p, _sz, ctypes.c_int, _p, _p], ctypes.c_int),
+    "pa_decode_store": ([_p, _p, _i64, _p, _p, _i64, _i64, _p, _p, _p, _p, _i32, _p, _i32, _i32,
+                         _i32, _i32, _i32, _i32, _i32, _f32, _i32, _p, _sz, ctypes.c_int, _p, _p],
+                        ctypes.c_int),
     "pa_decode_noalloc": ([_p, _p, _i64, _p, _p, _p, _i32, _p, _i32, _i32, _i32, _i32, _i32, _i32,
                            _i32, _f32, _i32, ctypes.c_int, _p, _p], ctypes.c_int),
     "pa_prefill_varlen": ([_p, _p, _i64, _p, _p, _p, _p, _i32, _i32, _i32, _p, _i32, _i32, _i32, _i32,
@@ -155,6 +158,41 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len, sca
                           int(partition_size), _ptr(workspace),
                           0 if workspace is None else workspace.numel() * workspace.element_size(),
                           PA_BF16, _ptr(err_flag), _stream()), "pa_decode")
+    return out
+
+
+def decode_store(q, key, value, k_cache, v_cache, slot_mapping, block_tables, context_lens,
+                 max_context_len, scale=None, out=None, workspace=None, partition_size=0,
+                 err_flag=None):
+    """One decode step's ``store_kvcache`` and ``decode`` in one launch (``pa_decode_store``):
+    key/value [B, Hkv, D] rows go to ``slot_mapping`` (the slots of each sequence's newest
+    position), then q [B, Hq, D] attends -> out [B, Hq, D] (bf16)."""
+    _need_cuda(q=q, key=key, value=value, k_cache=k_cache, v_cache=v_cache,
+               slot_mapping=slot_mapping, block_tables=block_tables, context_lens=context_lens,
+               out=out, workspace=workspace, err_flag=err_flag)
+    _need_bf16(q=q, key=key, value=value, k_cache=k_cache, v_cache=v_cache)
+    _need_i32(slot_mapping=slot_mapping, block_tables=block_tables, context_lens=context_lens)
+    nb, bs, hkv, d = k_cache.shape
+    B, hq, dq = q.shape
+    if dq != d:
+        raise ValueError("q head_dim differs from the pool's")
+    if key.shape[0] != B or value.shape[0] != B or slot_mapping.numel() != B:
+        raise ValueError("decode_store takes one new token per sequence")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, hq, d), dtype=torch.bfloat16, device=q.device)
+    ws_bytes = decode_workspace_size(B, hq, hkv, d, max_context_len, partition_size)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    _check(_lib.pa_decode_store(_ptr(out), _ptr(q), _token_stride(q, "q"), _ptr(key), _ptr(value),
+                                _token_stride(key, "key"), _token_stride(value, "value"),
+                                _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache),
+                                _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), B,
+                                int(max_context_len), hq, hkv, d, bs, nb, float(scale),
+                                int(partition_size), _ptr(workspace),
+                                0 if workspace is None else workspace.numel() * workspace.element_size(),
+                                PA_BF16, _ptr(err_flag), _stream()), "pa_decode_store")
     return out
 
 

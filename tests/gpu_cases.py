@@ -43,11 +43,26 @@ def pool_need(lens, bs):
 class DecodeCase(DecodeWorkload):
     """A decode workload plus the oracle's independent expectation."""
 
-    def run_gpu(self, partition_size=0, err_flag=None, poison=True):
+    def run_gpu(self, partition_size=0, err_flag=None, poison=True, fused=False):
+        """The decode step on the GPU: store_kvcache then decode, or (``fused``) both
+        through pa_decode_store in one launch.  Also keeps the output as ``self.out``."""
         self.upload(poison=poison)
-        out = self.step(err_flag=err_flag, partition_size=partition_size).clone()
+        if fused:
+            from paged_kv_attention_35_b200 import ops
+            ws = self.d_ws
+            need = ops.decode_workspace_size(self.B, self.hq, self.hkv, self.d,
+                                             self.max_context_len, partition_size)
+            if need > ws.numel():
+                ws = torch.empty(need, dtype=torch.uint8, device=self.d_out.device)
+            out = ops.decode_store(self.d_q, self.d_new_k, self.d_new_v, self.kc, self.vc,
+                                   self.d_slots, self.d_bt, self.d_cl, self.max_context_len,
+                                   out=self.d_out, workspace=ws, partition_size=partition_size,
+                                   err_flag=err_flag).clone()
+        else:
+            out = self.step(err_flag=err_flag, partition_size=partition_size).clone()
         torch.cuda.synchronize()
         self.bt_dev, self.cl_dev = self.d_bt, self.d_cl
+        self.out = out
         return out
 
     # ------------------------------------------------------------ oracle side
