@@ -25,11 +25,13 @@
 //    kernel stays bound by HBM.
 //  * positions >= context_len in the last tile are masked to -inf and their V
 //    rows zeroed in shared memory before P V (stale pool rows may hold NaN).
-//  * fused store (pa_decode_store): the CTA whose partition holds a
-//    sequence's newest position first writes that token's K and V rows of its
-//    KV head into the pool at slot_mapping[seq] (the store_kvcache of the
-//    step), orders the writes before its TMA reads with a proxy fence, and
-//    then streams as usual -- no other CTA of the launch reads that slot.
+//  * fused store (pa_decode_store): in the CTA whose partition holds a
+//    sequence's newest position, the consumer warp owning that position loads
+//    the token's new K and V rows of its KV head at the start, writes them to
+//    the pool at slot_mapping[seq] (the step's store_kvcache, for later steps)
+//    and, once the last tile has landed in shared memory, overwrites the stale
+//    row there -- no other CTA of the launch reads that slot, so no ordering
+//    between the global store and the TMA reads is needed.
 //  * the 4 warps merge (m, l, O) through shared memory; with one partition
 //    the CTA writes bf16 output, otherwise fp32 partials for the reduce kernel.
 
@@ -152,26 +154,6 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 
   if (warp == kDecWarps) {
     // ------------------------------------------------------------ producer
-    if (p.slots && t_end == L) {
-      // fused store of the newest token (position L-1) for this KV head
-      const int slot = __ldg(p.slots + seq);
-      const int lb = (L - 1) >> p.log2_bs;
-      const int bid = __ldg(p.block_tables + (int64_t)seq * p.max_blocks + lb);
-      if (slot >= 0 && bid >= 0 && bid < p.num_blocks &&
-          slot != bid * p.block_size + ((L - 1) & (p.block_size - 1)))
-        raise_flag(p.err_flag, PA_FLAG_SLOT_MISMATCH);
-      if (slot >= p.num_slots) raise_flag(p.err_flag, PA_FLAG_SLOT_OOB);
-      if (slot >= 0 && slot < p.num_slots) {
-        constexpr int C = D / 8;                   // 16-byte chunks per head row
-        const int64_t dst = ((int64_t)slot * p.hkv + kvh) * C;
-        const uint4 kx = __ldg(p.new_k + seq * p.new_k_stride16 + kvh * C + (lane & (C - 1)));
-        if (lane < C) p.kc[dst + lane] = kx;
-        const uint4 vx = __ldg(p.new_v + seq * p.new_v_stride16 + kvh * C + (lane & (C - 1)));
-        if (lane < C) p.vc[dst + lane] = vx;
-      }
-      fence_proxy_async_global();                  // the rows above precede this CTA's TMA reads
-    }
-    __syncwarp();
     if (lane == 0) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
@@ -238,12 +220,45 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   const int tw = warp * 16;
   const int mi = lane >> 3, ri = lane & 7;
 
+  // fused store: lanes 0..C-1 carry the K row's 16-byte chunks, C..2C-1 the V row's
+  constexpr int C = D / 8;
+  const int r_last = L - 1 - t_begin - (ntiles - 1) * kDecTile;   // newest position's tile row
+  bool patch = false;                              // this lane patches the last tile
+  uint4 nrow = make_uint4(0, 0, 0, 0);
+  if (p.slots && t_end == L && r_last >= tw && r_last < tw + 16) {
+    const int slot = __ldg(p.slots + seq);
+    const int bid = __ldg(p.block_tables + (int64_t)seq * p.max_blocks + ((L - 1) >> p.log2_bs));
+    const bool bid_ok = bid >= 0 && bid < p.num_blocks;
+    const int expect = bid * p.block_size + ((L - 1) & (p.block_size - 1));
+    const bool kv_lane = lane < 2 * C;
+    const bool is_v = lane >= C;
+    const int ch = lane % C;
+    if (kv_lane)
+      nrow = __ldg((is_v ? p.new_v + seq * p.new_v_stride16 : p.new_k + seq * p.new_k_stride16) +
+                   kvh * C + ch);
+    if (slot >= 0 && slot < p.num_slots) {
+      if (kv_lane) (is_v ? p.vc : p.kc)[((int64_t)slot * p.hkv + kvh) * C + ch] = nrow;
+      patch = kv_lane && bid_ok && slot == expect;
+      if (lane == 0 && bid_ok && slot != expect) raise_flag(p.err_flag, PA_FLAG_SLOT_MISMATCH);
+    } else if (slot >= p.num_slots && lane == 0) {
+      raise_flag(p.err_flag, PA_FLAG_SLOT_OOB);
+    }
+  }
+
   for (int it = 0; it < ntiles; ++it) {
     const int s = it % STAGES;
     if (!wait_or_abort(&full[s], (it / STAGES) & 1, abort_flag, p.err_flag)) break;
     const int valid = min(16, t_end - (t_begin + it * kDecTile + tw));
     uint8_t* kbase = smem + s * STAGE_BYTES;
     uint8_t* vbase = kbase + KV_BYTES;
+    if (patch && it == ntiles - 1) {
+      // the newest token's rows replace what the pool held at its position
+      const int ch = lane % C;
+      *reinterpret_cast<uint4*>((lane >= C ? vbase : kbase) + (ch >> 3) * HALF_BYTES +
+                                sw128(r_last, ch & 7)) = nrow;
+      fence_proxy_async_smem();                    // (the stage is not refilled: last tile)
+    }
+    __syncwarp();
     if (valid > 0) {
       if (valid < 16) {
         // zero V rows past the context (stale rows may be NaN; 0 * NaN = NaN)

@@ -10,8 +10,8 @@ seeded random id.
 
 One step: ``Scheduler.schedule()`` -> ``prepare_prefill`` / ``prepare_decode``
 -> one pinned host->device copy of the packed int32 metadata -> for every
-layer: ``store_kvcache`` of the step's new K/V rows into that layer's pool,
-then ``prefill_varlen`` or ``decode`` into a scratch output -> postprocess
+layer: ``store_kvcache`` of the step's new K/V rows into that layer's pool
+and ``prefill_varlen``, or both fused in ``decode_store``, into a scratch output -> postprocess
 (append tokens, finish, free).  All launches go to the current stream; the
 host runs ahead of the GPU except where it reuses a pinned staging buffer.
 
@@ -170,8 +170,8 @@ class Replay:
         for layer in range(c.num_layers):
             r = self.ring_index(step, layer)
             kc, vc = self.k_pools[layer], self.v_pools[layer]
-            ops.store_kvcache(self.k_ring[r, :nb], self.v_ring[r, :nb], kc, vc, slots)
-            ops.decode(self.q_ring[r, :nb], kc, vc, bt, cl, lb, out=out, workspace=self.g_ws)
+            ops.decode_store(self.q_ring[r, :nb], self.k_ring[r, :nb], self.v_ring[r, :nb], kc, vc,
+                             slots, bt, cl, lb, out=out, workspace=self.g_ws)
 
     def _decode_graph_step(self, md, n: int):
         """One decode step through a captured graph (see the module docstring)."""
@@ -253,13 +253,14 @@ class Replay:
         for layer in range(0 if (self.graphs and not is_prefill) else c.num_layers):
             r = self.ring_index(self.step_idx, layer)
             kc, vc = self.k_pools[layer], self.v_pools[layer]
-            ops.store_kvcache(self.k_ring[r, :n], self.v_ring[r, :n], kc, vc, slots)
             if is_prefill:
+                ops.store_kvcache(self.k_ring[r, :n], self.v_ring[r, :n], kc, vc, slots)
                 ops.prefill_varlen(self.q_ring[r, :n], kc, vc, cu_q, cu_k, md.max_seqlen_q,
                                    md.max_seqlen_k, bt, out=out)
             else:
-                ops.decode(self.q_ring[r, :n], kc, vc, bt, cl, md.max_context_len, out=out,
-                           workspace=self.ws)
+                # the step's store fused into the decode launch (pa_decode_store)
+                ops.decode_store(self.q_ring[r, :n], self.k_ring[r, :n], self.v_ring[r, :n], kc, vc,
+                                 slots, bt, cl, md.max_context_len, out=out, workspace=self.ws)
             if self.record == "all" or (self.step_idx, layer) in self.sample_at:
                 self.samples[(self.step_idx, layer)] = dict(
                     is_prefill=is_prefill, md=md, out=out.cpu().clone(),
@@ -271,7 +272,8 @@ class Replay:
         else:
             split = not is_prefill and ops.decode_workspace_size(
                 n, c.num_q_heads, c.num_kv_heads, c.head_dim, md.max_context_len) > 0
-        self.stats["launches"] += c.num_layers * (3 if split else 2)
+        # prefill: store + attention; decode: the fused store + decode, and the merge
+        self.stats["launches"] += c.num_layers * (2 if is_prefill else (2 if split else 1))
         if self.record:
             sm = md.slot_mapping.astype(np.int64)
             self.slot_writer[sm, 0] = self.step_idx
