@@ -161,18 +161,30 @@ def dist_setup():
 
 
 def max_over_ranks(torch, dist, world, x: float) -> float:
+    """The slowest rank's value (device-timed regions are reported as the max)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
+def whole_job_rate(world: int, units_per_rank_step: float, steps: int, max_total_ms: float) -> float:
+    """Replicas: every rank processes the same per-step work, so the whole job did
+    world x units x steps in the slowest rank's time; units per second."""
+    return world * units_per_rank_step * steps / (max_total_ms * 1e-3)
+
+
 def barrier(torch, dist, world):
-    torch.cuda.synchronize()
+    """Device work done, then every rank here (the CPU path for gloo ranks)."""
+    cuda = torch.cuda.is_available()
+    if cuda:
+        torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize()
+    if cuda:
+        torch.cuda.synchronize()
 
 
 # ------------------------------------------------------------ workloads (ours)
@@ -332,8 +344,8 @@ def ours(args):
     total_ms = max_over_ranks(torch, dist, world, r["step_ms_total"])
     step_ms = total_ms / args.steps
     step_bytes = w.step_bytes()
-    value = world * step_bytes * args.steps / (total_ms * 1e-3) / 1e9
-    tokens_s = world * w.B * args.steps / (total_ms * 1e-3)
+    value = whole_job_rate(world, step_bytes, args.steps, total_ms) / 1e9
+    tokens_s = whole_job_rate(world, w.B, args.steps, total_ms)
     kernel_gbs = step_bytes / (step_ms * 1e-3) / 1e9      # the step is the fused kernel (+ merge)
 
     e2e_ms, h2d, d2h = bench_decode_e2e(torch, w, args.steps, args.warmup, timer)
