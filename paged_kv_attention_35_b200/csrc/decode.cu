@@ -415,13 +415,32 @@ __global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeParams p) 
   const int n = (L + p.partition - 1) / p.partition;
   if (n <= 1) return;
   const int64_t base = ((int64_t)seq * p.hq + h) * p.max_splits;
-  float M = -INFINITY;
-  for (int s = 0; s < n; ++s) M = fmaxf(M, p.ws_ml[(base + s) * 2]);
-  float acc = 0.f, lsum = 0.f;
-  for (int s = 0; s < n; ++s) {
-    const float f = fast_exp2(p.ws_ml[(base + s) * 2] - M);
-    lsum += f * p.ws_ml[(base + s) * 2 + 1];
-    acc += f * p.ws_o[(base + s) * D + d];
+  // eight partitions per round, all their loads issued before any use (the
+  // kernel is latency-bound), merged online into (M, acc, lsum)
+  float M = -INFINITY, acc = 0.f, lsum = 0.f;
+  for (int s0 = 0; s0 < n; s0 += 8) {
+    float mv[8], lv[8], ov[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const bool v = s0 + k < n;
+      const int64_t sl = base + s0 + k;
+      mv[k] = v ? __ldcg(p.ws_ml + sl * 2) : -INFINITY;
+      lv[k] = v ? __ldcg(p.ws_ml + sl * 2 + 1) : 0.f;
+      ov[k] = v ? __ldcg(p.ws_o + sl * D + d) : 0.f;
+    }
+    float Mn = M;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) Mn = fmaxf(Mn, mv[k]);
+    const float a = M == -INFINITY ? 0.f : fast_exp2(M - Mn);
+    acc *= a;
+    lsum *= a;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float f = mv[k] == -INFINITY ? 0.f : fast_exp2(mv[k] - Mn);
+      acc += f * ov[k];
+      lsum += f * lv[k];
+    }
+    M = Mn;
   }
   p.out[((int64_t)seq * p.hq + h) * D + d] = __float2bfloat16(acc / lsum);
 }

@@ -168,3 +168,23 @@ def test_empty_batch_is_noop(cuda_device):
     out = ops.decode(q, kc, kc, torch.zeros(0, 1, dtype=torch.int32, device="cuda"),
                      torch.zeros(0, dtype=torch.int32, device="cuda"), 16)
     assert out.shape == (0, 4, 64)
+
+
+def test_store_full_size_permutation(cuda_device):
+    """The bench's bulk store at full size (65,536 rows, 8 x 128 bf16 each, slots a
+    seeded permutation of the whole pool): every pool row equals the input row the
+    permutation sends there -- bit-exact, checked through the inverse permutation."""
+    from paged_kv_attention_35_b200 import ops, synth
+    n, hkv, d, bs = 65536, 8, 128, 256
+    key = synth.bf16_normal((n, hkv, d), 7).cuda()
+    val = synth.bf16_normal((n, hkv, d), 8).cuda()
+    kc = torch.full((n // bs, bs, hkv, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    vc = torch.full_like(kc, float("nan"))
+    perm = synth.permutation(n, 9).astype(np.int64)
+    ops.store_kvcache(key, val, kc, vc, torch.from_numpy(perm.astype(np.int32)).cuda())
+    torch.cuda.synchronize()
+    inv = np.empty(n, np.int64)
+    inv[perm] = np.arange(n)
+    idx = torch.from_numpy(inv).cuda()
+    assert torch.equal(kc.view(n, hkv, d).view(torch.int16), key[idx].view(torch.int16))
+    assert torch.equal(vc.view(n, hkv, d).view(torch.int16), val[idx].view(torch.int16))
