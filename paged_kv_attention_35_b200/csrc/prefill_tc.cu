@@ -79,23 +79,6 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
   }
 }
 
-// 2^x on the FMA pipe, for a share of the softmax exponentials so the MUFU
-// unit is not the only one computing them (x <= 8 here; results below 2^-125
-// are returned as 0).  Cody-Waite split x = n + f, n = floor(x), f in [0, 1);
-// 2^f from a degree-3 minimax polynomial fitted (Remez exchange, relative
-// error) on [0, 1): max relative error 7.5e-5, far below bf16's half-ulp
-// (2^-9) -- P is rounded to bf16 right after; 2^n is added to the exponent.
-__device__ __forceinline__ float exp2_poly(float x) {
-  const float xc = fmaxf(x, -125.f);
-  const float n = floorf(xc);
-  const float f = xc - n;
-  float q = fmaf(0.07802452264047931f, f, 0.22606715542748335f);
-  q = fmaf(q, f, 0.6958335404947529f);
-  q = fmaf(q, f, 0.9999252185627155f);
-  const float r = __int_as_float(__float_as_int(q) + (static_cast<int>(n) << 23));
-  return x < -125.f ? 0.f : r;
-}
-
 // Packed / 3-input fp32 arithmetic of sm_100 (halves the softmax's issue slots).
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
@@ -121,31 +104,7 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   return d;
 }
 
-// Two exponentials per MUFU instruction: 2^x for a pair of fp32 arguments via
-// ex2.approx.f16x2.  The arguments are <= 8 (lazy rescale) and the results are
-// rounded to bf16 for P right after; the f16 argument's half-ulp error (at most
-// 2^-8 absolute for |x| < 16, i.e. 0.27% relative on p) is of the order of
-// that bf16 rounding, and x < -16 only reaches weights below 2^-16.
-// Off by default: the extra conversions cost more issue slots than the MUFU
-// time they save in this kernel (measured 454 vs 509 TFLOP/s on the
-// prefix-cached prefill workload); likewise the polynomial share below.
-#ifndef PA_EXP_F16X2
-#define PA_EXP_F16X2 0
-#endif
-__device__ __forceinline__ void exp2_pair_f16(float x0, float x1, float& e0, float& e1) {
-  uint32_t h, e;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(x1), "f"(x0));
-  asm("ex2.approx.f16x2 %0, %1;" : "=r"(e) : "r"(h));
-  asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
-      "cvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
-      : "=f"(e0), "=f"(e1)
-      : "r"(e));
-}
-
 constexpr int kBtCache = 256;    // block-table entries staged in shared memory
-#ifndef PA_EXP_POLY_OF_8
-#define PA_EXP_POLY_OF_8 0         // exponential pairs out of every 8 computed by exp2_poly
-#endif
 
 // Barrier block in shared memory (after the operand buffers).
 struct TcBars {
@@ -197,15 +156,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     return;
   }
   const int T = (q_len + kTcRows - 1) / kTcRows;   // query tiles of the sequence
-#ifdef PA_PAIR_FROM_START
-  const int tile_a = 2 * (gridDim.x - 1 - pp), tile_b = tile_a + 1;
-  if (tile_a >= T) return;
-  const bool hasB = tile_b < T;
-#else
   if (2 * pp >= T) return;
   const int tile_a = T - 1 - 2 * pp, tile_b = tile_a - 1;
   const bool hasB = tile_b >= 0;
-#endif
   const int q0A = tile_a * kTcRows;
   const int q0B = hasB ? tile_b * kTcRows : 0;
   const int cached = k_len - q_len;
@@ -431,18 +384,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int i = 0; i < kTcKeys; i += 2) {
         float x0, x1;
         f32x2_split(ffma2(f32x2(sv[i], sv[i + 1]), sc2, nm2), x0, x1);
-        // PA_EXP_POLY_OF_8 pairs in eight on the FMA pipe, the rest on MUFU
-        const bool poly = ((i >> 1) & 7) >= 8 - PA_EXP_POLY_OF_8;
-        float e0, e1;
-        if (poly) {
-          e0 = exp2_poly(x0);
-          e1 = exp2_poly(x1);
-        } else if (PA_EXP_F16X2) {
-          exp2_pair_f16(x0, x1, e0, e1);
-        } else {
-          e0 = fast_exp2(x0);
-          e1 = fast_exp2(x1);
-        }
+        const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
         rs2[(i >> 1) & 1] = fadd2(rs2[(i >> 1) & 1], f32x2(e0, e1));
         pk[i >> 1] = pack_bf16(e0, e1);
       }
