@@ -141,3 +141,27 @@ def test_python_binding_refuses_cpu_tensors(ops):
     pool = torch.zeros(4, 16, 8, 128, dtype=torch.bfloat16)
     with pytest.raises(TypeError):
         ops.store_kvcache(x, x, pool, pool, torch.zeros(2, dtype=torch.int32))
+
+
+def _decode_store(ops, **kw):
+    a = dict(out=256, q=256, qs=2048, key=512, value=512, ks=1024, vs=1024, slots=64, kc=256, vc=256,
+             bt=64, mb=16, cl=64, B=4, maxc=4096, hq=16, hkv=8, d=128, bs=256, nb=64, scale=0.088,
+             part=0, ws=None, wsb=0, dtype=0, flag=None)
+    a.update(kw)
+    return ops.lib().pa_decode_store(a["out"], a["q"], a["qs"], a["key"], a["value"], a["ks"], a["vs"],
+                                     a["slots"], a["kc"], a["vc"], a["bt"], a["mb"], a["cl"], a["B"],
+                                     a["maxc"], a["hq"], a["hkv"], a["d"], a["bs"], a["nb"], a["scale"],
+                                     a["part"], a["ws"], a["wsb"], a["dtype"], a["flag"], None)
+
+
+def test_decode_store_validation(ops):
+    assert _decode_store(ops, key=None) == 1                 # new rows missing
+    assert _decode_store(ops, slots=None) == 1
+    assert _decode_store(ops, value=520) == 1                # misaligned
+    assert _decode_store(ops, ks=100) == 1                   # stride < Hkv*D
+    assert _decode_store(ops, vs=1028) == 1                  # stride not a multiple of 8
+    assert _decode_store(ops, B=0, key=None, slots=None) == 0   # empty step: nothing to do
+    # the decode checks still apply, and a missing workspace is reported as for pa_decode
+    assert _decode_store(ops, hq=12, hkv=8) == 1
+    assert _decode_store(ops) == 3
+    assert "workspace" in ops.lib().pa_last_error_message().decode()
