@@ -277,14 +277,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       constexpr uint32_t idS = tc::idesc_bf16(kTcRows, kTcKeys, false, false);
       constexpr uint32_t idO = tc::idesc_bf16(kTcRows, 128, false, true);
       const int ntile[2] = {nA, nB};
+      // descriptors are built once; stepping K adds (byte offset / 16) to the
+      // start-address field (no carry: shared addresses stay below 256 KB)
+      const uint64_t dQ0 = tc::sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dK0 = tc::sdesc_sw128(smem_u32(sKV), 16, 1024);
+      const uint64_t dV0 = tc::sdesc_sw128(smem_u32(sKV), kHalf, 1024);
       auto issue_s = [&](int t, int j) {          // S_t(j) = Q_t K_j^T
         const int slot = (2 * j) % kRing;
-        const uint32_t aQ = smem_u32(sQ + t * kTile), aK = smem_u32(sKV + slot * kTile);
+        const uint64_t dQ = dQ0 + (uint64_t)((t * kTile) >> 4);
+        const uint64_t dK = dK0 + (uint64_t)((slot * kTile) >> 4);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t o = (ks >> 2) * kHalf + (ks & 3) * 32;
-          tc::mma_ss(tmem + 256 * t, tc::sdesc_sw128(aQ + o, 16, 1024),
-                     tc::sdesc_sw128(aK + o, 16, 1024), idS, ks > 0);
+          const uint64_t o = (uint64_t)(((ks >> 2) * kHalf + (ks & 3) * 32) >> 4);
+          tc::mma_ss(tmem + 256 * t, dQ + o, dK + o, idS, ks > 0);
         }
         tc::commit(&bar->s_full[t]);
       };
@@ -314,11 +319,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (j >= ntile[t]) continue;
           if (!tc_wait(&bar->p_full[t], j & 1, abort_flag, p.err_flag)) { ok = false; break; }
           tc::fence_after_sync();
-          const uint32_t aV = smem_u32(sKV + vslot * kTile);
+          const uint64_t dV = dV0 + (uint64_t)((vslot * kTile) >> 4);
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
             tc::mma_ts(tmem + 256 * t + 128, tmem + 256 * t + ks * 8,
-                       tc::sdesc_sw128(aV + ks * 2048, kHalf, 1024), idO, (j > 0 || ks > 0));
+                       dV + (uint64_t)((ks * 2048) >> 4), idO, (j > 0 || ks > 0));
           if (j == ntile[t] - 1) tc::commit(&bar->pv_done[t]);   // the epilogue waits on it
           if (j + 1 < ntile[t]) issue_s(t, j + 1);
         }
