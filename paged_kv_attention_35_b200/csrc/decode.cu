@@ -112,8 +112,12 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   uint64_t* empty = full + STAGES;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + STAGES);
 
+  // No early griddepcontrol.launch_dependents here: the dependent merge
+  // kernel's CTAs would become resident while this grid still has waves to
+  // run, holding registers that a second decode CTA per SM needs (measured
+  // 57.8 -> 56.5 us on the Qwen3-0.6B-shaped decode); it launches as this
+  // grid's CTAs exit.
   pdl_wait();
-  pdl_trigger();
   const int split = blockIdx.x;
   const int kvh = blockIdx.y / p.qtiles;
   const int qt = blockIdx.y % p.qtiles;
