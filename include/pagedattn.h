@@ -257,6 +257,18 @@ PA_API pa_status pa_prefill_varlen(void* out, const void* q, int64_t q_token_str
  */
 PA_API pa_status pa_watchdog_read(uint32_t* value);
 
+/*
+ * pa_selftest_wait_timeout -- health check of the failure detection: launches a
+ * one-thread kernel whose bounded mbarrier wait nothing completes; after
+ * limit_us microseconds (1 .. 2,000,000) it gives up, ORs PA_FLAG_TIMEOUT into
+ * *err_flag (device int32, may be NULL) and into the watchdog word, writes the
+ * nanoseconds it waited to *waited_ns (device uint64, may be NULL) and returns.
+ * The context stays usable.  The library's kernels bound every wait the same
+ * way (about two seconds).  Asynchronous on `stream`.
+ */
+PA_API pa_status pa_selftest_wait_timeout(int32_t* err_flag, uint32_t limit_us,
+                                          uint64_t* waited_ns, pa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

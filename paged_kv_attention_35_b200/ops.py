@@ -50,6 +50,7 @@ SIGNATURES = {
     "pa_prefill_varlen": ([_p, _p, _i64, _p, _p, _p, _p, _i32, _i32, _i32, _p, _i32, _i32, _i32, _i32,
                            _i32, _i32, _i32, _f32, ctypes.c_int, _p, _p], ctypes.c_int),
     "pa_watchdog_read": ([ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
+    "pa_selftest_wait_timeout": ([_p, ctypes.c_uint32, _p, _p], ctypes.c_int),
 }
 for _name, (_args, _res) in SIGNATURES.items():
     _fn = getattr(_lib, _name)
@@ -252,3 +253,13 @@ def watchdog_read() -> int:
     v = ctypes.c_uint32(0)
     _check(_lib.pa_watchdog_read(ctypes.byref(v)), "pa_watchdog_read")
     return int(v.value)
+
+
+def selftest_wait_timeout(limit_us: int = 50_000, err_flag=None, waited_ns=None) -> None:
+    """Health check of the failure detection (``pa_selftest_wait_timeout``): a bounded
+    wait that nothing completes gives up after ``limit_us`` and reports PA_FLAG_TIMEOUT
+    in ``err_flag`` (device int32) and the watchdog word; ``waited_ns`` (device int64)
+    receives the time it waited."""
+    _need_cuda(err_flag=err_flag, waited_ns=waited_ns)
+    _check(_lib.pa_selftest_wait_timeout(_ptr(err_flag), int(limit_us), _ptr(waited_ns), _stream()),
+           "pa_selftest_wait_timeout")

@@ -165,3 +165,8 @@ def test_decode_store_validation(ops):
     assert _decode_store(ops, hq=12, hkv=8) == 1
     assert _decode_store(ops) == 3
     assert "workspace" in ops.lib().pa_last_error_message().decode()
+
+
+def test_selftest_validation(ops):
+    assert ops.lib().pa_selftest_wait_timeout(None, 0, None, None) == 1
+    assert ops.lib().pa_selftest_wait_timeout(None, 3_000_000, None, None) == 1

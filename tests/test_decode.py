@@ -188,3 +188,21 @@ def test_store_full_size_permutation(cuda_device):
     idx = torch.from_numpy(inv).cuda()
     assert torch.equal(kc.view(n, hkv, d).view(torch.int16), key[idx].view(torch.int16))
     assert torch.equal(vc.view(n, hkv, d).view(torch.int16), val[idx].view(torch.int16))
+
+
+def test_bounded_wait_gives_up_and_reports(cuda_device):
+    """Failure detection: a wait nothing completes gives up after its limit, reports
+    PA_FLAG_TIMEOUT in err_flag and in the watchdog word, and the context stays
+    usable (a decode step right after is checked against the oracle)."""
+    from paged_kv_attention_35_b200 import ops
+    ops.watchdog_read()                                      # clear
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    waited = torch.zeros(1, dtype=torch.int64, device="cuda")
+    ops.selftest_wait_timeout(50_000, err, waited)
+    torch.cuda.synchronize()
+    assert int(err.item()) & ops.FLAG_TIMEOUT
+    assert 50e6 <= int(waited.item()) < 2e9
+    assert ops.watchdog_read() & ops.FLAG_TIMEOUT
+    assert ops.watchdog_read() == 0                          # read clears it
+    c = DecodeCase([17, 64, 100, 255], hq=4, hkv=2, d=64, bs=16, num_blocks=64, seed=1001)
+    compare(c.run_gpu(), c.oracle_decode(), "decode after a timed-out wait")
