@@ -1,24 +1,30 @@
 #!/usr/bin/env python
 """Benchmark of the paged-KV attention hot path on B200.
 
-Default (N=1): one layer of Qwen3-0.6B-shaped decode -- batch 32, context
-lengths uniform in [128, 4096], 16 query / 8 KV heads, head_dim 128, block
-size 256, shuffled pool sized 1.25x the need.  One step = store each
-sequence's new K/V row into the pool + paged decode attention over the batch.
+Default (N=1): one layer of 7B-GQA-shaped decode -- batch 256, context
+lengths uniform in [512, 4096], 28 query / 4 KV heads, head_dim 128, block
+size 256, shuffled pool sized 1.25x the need (the largest decode
+configuration).  One step = store each sequence's new K/V row into the pool +
+paged decode attention over the batch (one fused launch, then the split-K
+merge).
 
 Metric: decode-step KV GB/s (algorithmic bytes of the step / step time), with
 tokens/s (sequences decoded per second for this layer) beside it.  Inputs are
 resident in HBM when timing starts; L2 is flushed (a 512 MiB write, then a
-512 MiB read so the write's dirty lines are gone too) before every timed step and each step is bracketed by CUDA events on the launching
-stream.  With --gpus N (torchrun, one rank per GPU) every rank runs its own
-replica of the workload (no collective on the data path: "scaling": "weak")
-and the time is the max over ranks.
+512 MiB read so the write's dirty lines are gone too) before every timed step
+and each step is bracketed by CUDA events on the launching stream.  With
+--gpus N (torchrun, one rank per GPU) every rank runs its own replica of the
+workload (no collective on the data path: "scaling": "weak") and the time is
+the max over ranks.
 
-Also measured in the same run and reported under "workloads": 7B-GQA decode
-(batch 256, 28/4 heads, block 256 and block 16), the prefix-cached prefill
-(TFLOP/s), a large store_kvcache (GB/s) and the continuous-batching trace
-replay (tokens/s).  ``--impl reference`` times the CPU oracle on a bounded
-sample of the same workload instead.
+Also measured in the same run, at the same --steps / --warmup, and reported
+under "workloads": Qwen3-0.6B-shaped decode (batch 32, 16/8 heads), the
+7B-GQA decode at block 16, the prefix-cached prefill (TFLOP/s), a large
+store_kvcache (GB/s) and the continuous-batching trace replay (tokens/s, with
+GPU-busy and host control-plane time).  "cpu_baselines" times the CPU oracle
+on every configuration (bounded samples; the trace replay's full-trace figure
+is a labelled projection).  ``--impl reference`` times the CPU oracle on a
+bounded sample of the headline workload instead.
 """
 
 from __future__ import annotations
@@ -330,6 +336,20 @@ def bench_store_large(torch, steps, warmup, timer):
     return nbytes, ms
 
 
+def decode_config(spec, w, partition, world):
+    """The `config` object of a decode bench line (both arms print the same one)."""
+    lo, hi = (spec.ctx_lo, spec.ctx_hi) if not spec.fixed_lens else (min(w.lens), max(w.lens))
+    return {"workload": spec.name, "num_seqs": w.B, "context_lens": f"U[{lo},{hi}]",
+            "sum_context": int(sum(w.lens)), "num_q_heads": w.hq, "num_kv_heads": w.hkv,
+            "head_dim": w.d, "block_size": w.bs, "num_blocks": w.nb,
+            "partition": partition or "auto",
+            "l2": "flushed before every step (512 MiB write, then 512 MiB read)",
+            "parallelism": f"replicas x{world}"}
+
+
+METRIC = "paged decode attention KV GB/s (decode step: store_kvcache + decode)"
+
+
 def ours(args):
     torch, dist, world, rank, local = dist_setup()
     from paged_kv_attention_35_b200 import ops  # noqa: F401  (fails loudly without the library)
@@ -361,14 +381,15 @@ def ours(args):
     if not args.quick and rank == 0:
         extra = secondary(torch, args, timer, pk)
 
-    cpu = None
+    cpu, cpus = None, None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline_decode(w, budget_s=args.cpu_budget)
+        cpus = cpu_baselines(args, w, extra)
 
     if rank == 0:
         traffic = load_traffic("decode_kernel", args.workload)
         line = {
-            "metric": "paged decode attention KV GB/s (decode step: store_kvcache + decode)",
+            "metric": METRIC,
             "value": round(value, 1),
             "unit": "GB/s",
             "n_gpus": world,
@@ -380,11 +401,7 @@ def ours(args):
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16 K/V/q, seeded context lengths and shuffled pool)",
-            "config": {"workload": spec.name, "num_seqs": w.B, "context_lens": "U[128,4096]",
-                       "sum_context": int(sum(w.lens)), "num_q_heads": w.hq, "num_kv_heads": w.hkv,
-                       "head_dim": w.d, "block_size": w.bs, "num_blocks": w.nb,
-                       "partition": args.partition or "auto", "l2": "flushed before every step (512 MiB write, then 512 MiB read)",
-                       "parallelism": f"replicas x{world}"},
+            "config": decode_config(spec, w, args.partition, world),
             "tokens_per_s": round(tokens_s, 1),
             "breakdown_ms": {"fused_store_decode": round(r["step_ms"], 4),
                              "store_then_decode": round(r["two_launch_ms"], 4),
@@ -401,6 +418,7 @@ def ours(args):
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
+            "cpu_baselines": cpus,
             "workloads": extra,
             "pages_context": {"qwen7b_tokens_per_s": {"bs1": 32, "bs8": 215, "bs16": 398},
                               "note": "end-to-end model throughput quoted by the pages, hardware not stated"},
@@ -412,23 +430,29 @@ def ours(args):
 
 
 def secondary(torch, args, timer, pk):
-    """The other workloads, each at its own roofline (rank 0, N=1 or any N)."""
+    """The other workloads, each at its own roofline (rank 0), at the same --steps / --warmup."""
     from paged_kv_attention_35_b200 import synth
     from paged_kv_attention_35_b200.workloads import DecodeWorkload
     out = {}
-    steps = max(3, min(args.steps, 10))
-    for bs in (256, 16):
-        w = DecodeWorkload.from_spec(synth.WORKLOADS["gqa7b_decode"], block_size=bs).upload("cuda")
-        r = bench_decode(torch, w, steps, 3, timer)
+    steps, warm = args.steps, args.warmup
+    others = [("qwen3_0p6b_decode", None), ("gqa7b_decode", 256), ("gqa7b_decode", 16)]
+    for name, bs in others:
+        spec = synth.WORKLOADS[name]
+        if name == args.workload and bs in (None, spec.block_size):
+            continue                               # the headline itself
+        w = DecodeWorkload.from_spec(spec, block_size=bs).upload("cuda")
+        r = bench_decode(torch, w, steps, warm, timer)
+        step_gbs = w.step_bytes() / (r["step_ms"] * 1e-3) / 1e9
         gbs = w.kv_bytes() / (r["decode_ms"] * 1e-3) / 1e9
-        out[f"gqa7b_decode_bs{bs}"] = {
+        out[f"{name}_bs{w.bs}"] = {
             "step_ms": round(r["step_ms"], 4), "decode_ms": round(r["decode_ms"], 4),
             "store_then_decode_ms": round(r["two_launch_ms"], 4), "kv_bytes": w.kv_bytes(),
+            "step_GBs": round(step_gbs, 1), "frac_hbm_step": round(step_gbs / pk["hbm_gbs"], 4),
             "decode_GBs": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4),
             "tokens_per_s": round(w.B / (r["step_ms"] * 1e-3), 1)}
         del w
         torch.cuda.empty_cache()
-    w, store_ms, attn_ms = bench_prefill(torch, steps, 3, timer)
+    w, store_ms, attn_ms = bench_prefill(torch, steps, warm, timer)
     tf = w.flops() / (attn_ms * 1e-3) / 1e12
     out["prefix_prefill"] = {
         "attn_ms": round(attn_ms, 4), "store_ms": round(store_ms, 4), "flops": w.flops(),
@@ -438,20 +462,19 @@ def secondary(torch, args, timer, pk):
         "store_GBs": round(w.store_bytes() / (store_ms * 1e-3) / 1e9, 1)}
     del w
     torch.cuda.empty_cache()
-    nbytes, ms = bench_store_large(torch, steps, 3, timer)
+    nbytes, ms = bench_store_large(torch, steps, warm, timer)
     out["store_kvcache_65536"] = {"ms": round(ms, 4), "bytes": nbytes,
                                   "GBs": round(nbytes / (ms * 1e-3) / 1e9, 1),
                                   "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
     torch.cuda.empty_cache()
     if not args.no_replay:
-        try:
-            from paged_kv_attention_35_b200.replay import run_replay_bench
-            out["trace_replay"] = run_replay_bench(torch, max_steps=args.replay_steps, graphs=False)
-            g = run_replay_bench(torch, max_steps=args.replay_steps, graphs=True)
-            out["trace_replay_graphs"] = {k: g[k] for k in (
-                "tokens_per_s", "wall_s", "steps", "graph_steps", "graph_captures", "decode_kv_GBs")}
-        except ImportError:
-            pass
+        from paged_kv_attention_35_b200.replay import run_replay_bench
+        out["trace_replay"] = run_replay_bench(torch, max_steps=args.replay_steps, graphs=False)
+        g = run_replay_bench(torch, max_steps=args.replay_steps, graphs=True)
+        out["trace_replay_graphs"] = {k: g[k] for k in (
+            "tokens_per_s", "wall_s", "gpu_busy_s", "host_s", "steps", "graph_steps",
+            "graph_captures", "decode_kv_GBs")}
+        torch.cuda.empty_cache()
     return out
 
 
@@ -561,6 +584,138 @@ def _blas_threads(default):
     return default
 
 
+def cpu_baselines(args, w3, extra):
+    """The oracle (as it stands, never tuned) timed on every configuration on this
+    host's cores.  Decode configs: bounded samples with all BLAS threads and with one;
+    the prefix-cached prefill: the whole workload once; the trace replay: sampled
+    (step, layer) pairs of a recorded replay, projected to the whole trace by the
+    number of (query, key) pairs it visits (labelled as a projection)."""
+    from threadpoolctl import threadpool_limits
+    from paged_kv_attention_35_b200 import synth
+    from paged_kv_attention_35_b200.workloads import DecodeWorkload
+    budget = max(1.0, args.cpu_budget / 3)
+    res = {}
+    tiny = DecodeWorkload.from_spec(synth.WORKLOADS["tiny_decode"])
+    w2 = DecodeWorkload.from_spec(synth.WORKLOADS["qwen3_0p6b_decode"])
+    for name, w, b in (("tiny_decode", tiny, 1.0), ("qwen3_0p6b_decode", w2, budget),
+                       ("gqa7b_decode", w3, budget)):
+        e = {}
+        if name != "gqa7b_decode" or w3.bs != 256:
+            e["all_threads"] = cpu_baseline_decode(w, budget_s=b)
+        with threadpool_limits(limits=1):
+            e["one_thread"] = cpu_baseline_decode(w, budget_s=b)
+        e["one_thread"]["cores"] = 1
+        res[name] = e
+    res["prefix_prefill"] = cpu_baseline_prefill()
+    rp = extra.get("trace_replay") if extra else None
+    if rp and not args.no_replay:
+        res["trace_replay"] = cpu_baseline_replay(rp, budget_s=budget)
+    return res
+
+
+def cpu_baseline_prefill():
+    """The oracle on the whole prefix-cached prefill (16 sequences, every head)."""
+    import oracle
+    from paged_kv_attention_35_b200 import synth
+    from paged_kv_attention_35_b200.workloads import PrefixPrefillWorkload
+    w = PrefixPrefillWorkload(seed=synth.SEED_BASE + 4)
+    q, kp, vp, cu_q, cu_k, bt = prefill_oracle_inputs(w)
+    t0 = time.perf_counter()
+    oracle.ref_prefill(q, kp, vp, cu_q, cu_k, bt)
+    dt = time.perf_counter() - t0
+    return {"value": round(w.flops() / dt / 1e12, 6), "unit": "TFLOP/s",
+            "cores": _blas_threads(len(os.sched_getaffinity(0))), "kind": "oracle",
+            "sample": f"the whole workload: {len(w.seqs)} sequences, {int(w.md.total_q)} queries x "
+                      f"{w.hq} heads, oracle time {dt:.2f} s", "seconds": round(dt, 2)}
+
+
+def prefill_oracle_inputs(w, seqs=None):
+    """Oracle inputs (float64) of a prefix-cached prefill workload: packed q and a compact
+    pool holding the listed sequences' logical K/V (renumbered blocks)."""
+    import oracle
+    import torch
+
+    def bits(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    seqs = list(range(len(w.seqs))) if seqs is None else list(seqs)
+    k_lens = [w.k_lens[i] for i in seqs]
+    nblk = [-(-L // w.bs) for L in k_lens]
+    bt = np.full((len(seqs), max(nblk)), -1, np.int32)
+    kp = np.zeros((sum(nblk), w.bs, w.hkv, w.d), np.uint16)
+    vp = np.zeros_like(kp)
+    k = 0
+    for j, i in enumerate(seqs):
+        bt[j, :nblk[j]] = np.arange(k, k + nblk[j])
+        kp[k:k + nblk[j]].reshape(-1, w.hkv, w.d)[:k_lens[j]] = bits(w.k[i])
+        vp[k:k + nblk[j]].reshape(-1, w.hkv, w.d)[:k_lens[j]] = bits(w.v[i])
+        k += nblk[j]
+    cu = w.md.cu_seqlens_q
+    qall = oracle.bf16_bits_to_f64(bits(w.q))
+    q = np.concatenate([qall[cu[i]:cu[i + 1]] for i in seqs])
+    cu_q = np.concatenate([[0], np.cumsum([w.q_lens[i] for i in seqs])])
+    cu_k = np.concatenate([[0], np.cumsum(k_lens)])
+    return q, oracle.bf16_bits_to_f64(kp), oracle.bf16_bits_to_f64(vp), cu_q, cu_k, bt
+
+
+def cpu_baseline_replay(stats, budget_s=10.0):
+    """Oracle time for sampled sequences of sampled (step, layer) pairs of the trace
+    replay, and a projection to the whole trace by visited (query, key) pairs."""
+    import oracle
+    import torch
+    from paged_kv_attention_35_b200.replay import Replay, ReplayConfig
+
+    def bits(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    cfg = ReplayConfig()
+    rp = Replay(cfg, record=True)
+    last = cfg.num_layers - 1
+    rp.sample_at = {(0, 0), (1, last), (3, 0), (40, last), (120, 0)}
+    rp.run(max_steps=121)
+    torch.cuda.synchronize()
+    f64 = oracle.bf16_bits_to_f64
+    spent = {"prefill": [0.0, 0], "decode": [0.0, 0]}      # seconds, visited pairs x heads
+    for (step, layer), smp in sorted(rp.samples.items()):
+        snap = rp.snap[step]
+        md = smp["md"]
+        q_all = f64(bits(rp.q_ring_cpu[rp.ring_index(step, layer)]))
+        kind = "prefill" if smp["is_prefill"] else "decode"
+        for j in range(min(len(smp["lens"]), 4)):
+            if spent[kind][0] > budget_s / 2:
+                break
+            bt, L = smp["block_tables"][j], smp["lens"][j]
+            slots = oracle.ref_slot_mapping(bt, range(L), cfg.block_size)
+            wr = snap[slots]
+            K = f64(np.stack([bits(rp.k_ring_cpu[rp.ring_index(int(a), layer)][int(b)]) for a, b in wr]))
+            V = f64(np.stack([bits(rp.v_ring_cpu[rp.ring_index(int(a), layer)][int(b)]) for a, b in wr]))
+            kp, vp = K[None], V[None]
+            t0 = time.perf_counter()
+            if kind == "prefill":
+                a, b = int(md.cu_seqlens_q[j]), int(md.cu_seqlens_q[j + 1])
+                oracle.ref_prefill(q_all[a:b], kp, vp, [0, b - a], [0, L], np.array([[0]]))
+                pairs = (b - a) * (L - (b - a)) + (b - a) * (b - a + 1) // 2
+            else:
+                oracle.ref_decode(q_all[j:j + 1], kp, vp, np.array([[0]]), [L])
+                pairs = L
+            spent[kind][0] += time.perf_counter() - t0
+            spent[kind][1] += pairs * cfg.num_q_heads
+    per = {k: (v[0] / v[1] if v[1] else None) for k, v in spent.items()}
+    total_pairs = {"prefill": stats["prefill_pairs"] * cfg.num_layers * cfg.num_q_heads,
+                   "decode": stats["decode_context_tokens"] * cfg.num_layers * cfg.num_q_heads}
+    proj = sum(per[k] * total_pairs[k] for k in per if per[k] is not None)
+    tokens = stats["prefill_tokens"] + stats["decode_tokens"]
+    return {"value": round(tokens / proj, 3) if proj else None, "unit": "tokens/s",
+            "cores": _blas_threads(len(os.sched_getaffinity(0))), "kind": "oracle",
+            "projection": True,
+            "sample": (f"sampled sequences of (step, layer) pairs {sorted(rp.samples)} of the "
+                       f"replayed trace: prefill {spent['prefill'][0]:.2f} s for "
+                       f"{spent['prefill'][1]} (query, key, head) triples, decode "
+                       f"{spent['decode'][0]:.2f} s for {spent['decode'][1]}; PROJECTED to the "
+                       f"whole trace's {total_pairs['prefill']} + {total_pairs['decode']} triples "
+                       f"({proj:.0f} s)" if proj else "no sample")}
+
+
 def reference(args):
     """The oracle as the reference arm: same metric/config, bounded sample per step."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -581,12 +736,11 @@ def reference(args):
         vals.append(last["value"])
     v = float(np.mean(vals))
     line = {
-        "impl": "reference", "metric": "paged decode attention KV GB/s (decode step: store_kvcache + decode)",
+        "impl": "reference", "metric": METRIC,
         "value": round(v, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (same seeded workload)",
-        "config": {"workload": spec.name, "num_seqs": w.B, "num_q_heads": w.hq,
-                   "num_kv_heads": w.hkv, "head_dim": w.d, "block_size": w.bs},
+        "config": decode_config(spec, w, args.partition, world),
         "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "kind": "oracle",
                          "cores": last["cores"], "sample": last["sample"]},
         "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -600,7 +754,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="qwen3_0p6b_decode")
+    ap.add_argument("--workload", default="gqa7b_decode")
     ap.add_argument("--partition", type=int, default=0)
     ap.add_argument("--quick", action="store_true", help="primary workload only")
     ap.add_argument("--no-cpu", action="store_true")

@@ -204,8 +204,10 @@ PA_API pa_status pa_decode_store(void* out, const void* q, int64_t q_token_strid
  *     scratch are rejected with PA_ERR_WORKSPACE before any launch; a larger
  *     partition_size shrinks the need.
  *   - The first call on each device (with that device current) looks up the
- *     scratch array's device address once (cudaGetSymbolAddress); make that
- *     first call before any stream capture.
+ *     scratch array's device address (cudaGetSymbolAddress) and remembers it
+ *     for that device's context; make that first call before any stream
+ *     capture.  A context re-created later (cudaDeviceReset) is noticed by its
+ *     id and the address is looked up again.
  *   - Every call shares the one array, which keeps the last call's contents
  *     (nothing in it needs to start at zero).  Calls that overlap on the GPU --
  *     on two streams at once, or from two host threads -- race on it.

@@ -241,10 +241,14 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       nrow = __ldg((is_v ? p.new_v + seq * p.new_v_stride16 : p.new_k + seq * p.new_k_stride16) +
                    kvh * C + ch);
     if (slot >= 0 && slot < p.num_slots) {
-      if (kv_lane) (is_v ? p.vc : p.kc)[((int64_t)slot * p.hkv + kvh) * C + ch] = nrow;
+      // with a group of more than 16 query heads several CTAs (q tiles) share
+      // this KV head: the first writes the pool row, every one patches its own
+      // landed tile (no CTA of this launch reads the row back from the pool)
+      if (kv_lane && qt == 0) (is_v ? p.vc : p.kc)[((int64_t)slot * p.hkv + kvh) * C + ch] = nrow;
       patch = kv_lane && bid_ok && slot == expect;
-      if (lane == 0 && bid_ok && slot != expect) raise_flag(p.err_flag, PA_FLAG_SLOT_MISMATCH);
-    } else if (slot >= p.num_slots && lane == 0) {
+      if (lane == 0 && qt == 0 && bid_ok && slot != expect)
+        raise_flag(p.err_flag, PA_FLAG_SLOT_MISMATCH);
+    } else if (slot >= p.num_slots && lane == 0 && qt == 0) {
       raise_flag(p.err_flag, PA_FLAG_SLOT_OOB);
     }
   }
@@ -455,17 +459,16 @@ static pa_status launch_decode_d(const DecodeArgs& a, const CUtensorMap& mk, con
   constexpr int HALVES = D / 64;
   constexpr int STAGE_BYTES = 2 * HALVES * kDecTile * 128;
   const size_t smem = (size_t)kDecStages * STAGE_BYTES + 1024 + 2 * kDecStages * 8 + 16;
-  static bool attr_done = false;      // benign race: idempotent attribute set
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, kDecStages>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return cuda_fail(e, "decode smem attribute");
-    attr_done = true;
-  }
+  pa_status s = ensure_smem_attr((const void*)decode_kernel<D, kDecStages>, (int)smem,
+                                 "decode smem attribute");
+  if (s != PA_OK) return s;
   dim3 grid(a.max_splits, a.hkv * prm.qtiles, a.num_seqs);
   cudaError_t e = launch_pdl(decode_kernel<D, kDecStages>, grid, dim3(kDecThreads), smem, a.stream,
                              mk, mv, prm);
-  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  if (e != cudaSuccess) {
+    forget_smem_attr((const void*)decode_kernel<D, kDecStages>);
+    return cuda_fail(e, "decode launch");
+  }
   if (a.max_splits > 1) {
     e = launch_pdl(decode_reduce_kernel<D>, dim3(a.hq, a.num_seqs), dim3(D), 0, a.stream, prm);
     if (e != cudaSuccess) return cuda_fail(e, "decode reduce launch");

@@ -13,14 +13,16 @@
 // every GPU that loads the library holds until the process exits.
 //
 // Host code cannot use the array's name as a device address (in host code it
-// is only a stand-in symbol), so the first call on each device, with that
-// device current, asks the runtime for the array's device address
-// (cudaGetSymbolAddress) and remembers it for that device.  After that the
-// call is pa_decode with the scratch in place of the caller's workspace.  All
-// calls share the one array and it keeps whatever the last call left in it:
-// nothing there has to start at zero (the decode writes every partial before
-// its merge reads it), but calls that overlap on the GPU -- two streams, or
-// two host threads launching at once -- race on it.
+// is only a stand-in symbol), so the first call in each CUDA context -- once
+// per device, with that device current -- asks the runtime for the array's
+// device address (cudaGetSymbolAddress) and remembers it together with the
+// context's unique id; a call from a context re-created since (after
+// cudaDeviceReset, say) finds a different id and looks the address up again.
+// After that the call is pa_decode with the scratch in place of the caller's
+// workspace.  All calls share the one array and it keeps whatever the last
+// call left in it: nothing there has to start at zero (the decode writes every
+// partial before its merge reads it), but calls that overlap on the GPU -- two
+// streams, or two host threads launching at once -- race on it.
 
 #include <mutex>
 
@@ -34,23 +36,59 @@ static __device__ __align__(256) unsigned char g_decode_scratch[PA_DECODE_NOALLO
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices];   // device address of g_decode_scratch, per device
+struct ScratchAddr {
+  unsigned long long ctx_id;   // cuCtxGetId of the context the address belongs to
+  void* addr;                  // device address of g_decode_scratch there
+};
+ScratchAddr g_scratch[kMaxDevices];
 
-// Device address of the scratch array on the current device (looked up once per device).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (0 if it cannot be read).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &f, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(f);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx &&
+      get_id(ctx, &id) == CUDA_SUCCESS)
+    return id;
+  return 0;
+}
+
+// Device address of the scratch array in the current device's context.
 pa_status scratch_address(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(PA_ERR_UNSUPPORTED, "device ordinal >= 64");
+  // 0 when no context is current yet: the lookup below then makes the
+  // device's primary context current, and its id is read afterwards
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  ScratchAddr& c = g_scratch[dev];
+  if (c.addr == nullptr || ctx == 0 || c.ctx_id != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(decode scratch)");
     if (p == nullptr) return fail(PA_ERR_CUDA, "cudaGetSymbolAddress returned NULL");
-    g_scratch_addr[dev] = p;
+    c.addr = p;
+    c.ctx_id = ctx ? ctx : current_context_id();
   }
-  *out = g_scratch_addr[dev];
+  *out = c.addr;
   return PA_OK;
 }
 

@@ -21,12 +21,49 @@ __device__ unsigned int g_watchdog = 0;
 
 static thread_local std::string t_last_error;
 
-bool pdl_enabled() {
-  static const bool on = [] {
-    const char* e = getenv("PA_PDL");
-    return !(e && e[0] == '0');
-  }();
-  return on;
+// ------------------------------------------------- per-device launch state
+namespace {
+constexpr int kMaxDev = 64;
+std::mutex g_dev_mu;
+std::unordered_map<const void*, uint64_t> g_attr_done;   // kernel -> bitmask of devices
+int g_sm_count[kMaxDev];
+}  // namespace
+
+pa_status ensure_smem_attr(const void* kernel, int bytes, const char* what) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  const uint64_t bit = dev < kMaxDev ? (uint64_t)1 << dev : 0;
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    auto it = g_attr_done.find(kernel);
+    if (bit && it != g_attr_done.end() && (it->second & bit)) return PA_OK;
+  }
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  g_attr_done[kernel] |= bit;
+  return PA_OK;
+}
+
+void forget_smem_attr(const void* kernel) {
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  g_attr_done.erase(kernel);
+}
+
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return 148;
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (g_sm_count[dev] > 0) return g_sm_count[dev];
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  g_sm_count[dev] = n;
+  return n;
 }
 
 pa_status fail(pa_status s, const std::string& msg) {
@@ -63,10 +100,10 @@ struct MapKey {
   int64_t rows;
   int heads, d;
   int64_t stride;
-  int box;
+  int box, box_heads;
   bool operator==(const MapKey& o) const {
     return base == o.base && rows == o.rows && heads == o.heads && d == o.d && stride == o.stride &&
-           box == o.box;
+           box == o.box && box_heads == o.box_heads;
   }
 };
 struct MapKeyHash {
@@ -74,6 +111,7 @@ struct MapKeyHash {
     size_t h = std::hash<const void*>()(k.base);
     h ^= std::hash<int64_t>()(k.rows * 1315423911ll + k.stride) + 0x9e3779b97f4a7c15ull + (h << 6);
     h ^= std::hash<int64_t>()((int64_t)k.heads << 40 | (int64_t)k.d << 20 | k.box) + (h << 6);
+    h ^= std::hash<int>()(k.box_heads) + (h << 3);
     return h;
   }
 };
@@ -82,8 +120,8 @@ static std::mutex g_map_mu;
 static std::unordered_map<MapKey, CUtensorMap, MapKeyHash> g_maps;
 
 pa_status get_tensor_map(CUtensorMap* out, const void* base, int64_t rows, int heads, int head_dim,
-                         int64_t row_stride_elems, int box_rows) {
-  MapKey key{base, rows, heads, head_dim, row_stride_elems, box_rows};
+                         int64_t row_stride_elems, int box_rows, int box_heads) {
+  MapKey key{base, rows, heads, head_dim, row_stride_elems, box_rows, box_heads};
   {
     std::lock_guard<std::mutex> lk(g_map_mu);
     auto it = g_maps.find(key);
@@ -96,7 +134,7 @@ pa_status get_tensor_map(CUtensorMap* out, const void* base, int64_t rows, int h
   if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)heads, (cuuint64_t)rows};
   cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2, (cuuint64_t)row_stride_elems * 2};
-  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
   cuuint32_t estr[3] = {1, 1, 1};
   CUtensorMap m;
   CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
@@ -104,8 +142,9 @@ pa_status get_tensor_map(CUtensorMap* out, const void* base, int64_t rows, int h
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     char buf[160];
-    snprintf(buf, sizeof buf, "cuTensorMapEncodeTiled failed (%d) rows=%lld heads=%d d=%d box=%d",
-             (int)r, (long long)rows, heads, head_dim, box_rows);
+    snprintf(buf, sizeof buf,
+             "cuTensorMapEncodeTiled failed (%d) rows=%lld heads=%d d=%d box=%d x %d heads", (int)r,
+             (long long)rows, heads, head_dim, box_rows, box_heads);
     return fail(PA_ERR_CUDA, buf);
   }
   {
@@ -151,7 +190,7 @@ int decode_auto_partition(int num_seqs, int num_kv_heads, int max_context_len) {
   return (int)p;
 }
 
-static void decode_ws_layout(int num_seqs, int hq, int d, int splits, size_t* o_bytes,
+static void decode_ws_layout(int num_seqs, int hq, int d, int64_t splits, size_t* o_bytes,
                              size_t* ml_bytes) {
   size_t rows = (size_t)num_seqs * hq * splits;
   *o_bytes = (rows * d * sizeof(float) + 255) / 256 * 256;
@@ -217,8 +256,8 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t n
   int p = partition_size > 0 ? partition_size
                              : decode_auto_partition(num_seqs, num_kv_heads, max_context_len);
   if (p <= 0 || p % 64) return 0;
-  int splits = (max_context_len + p - 1) / p;
-  if (splits <= 1) return 0;
+  const int64_t splits = ((int64_t)max_context_len + p - 1) / p;
+  if (splits <= 1 || splits > 65535) return 0;
   size_t ob, mb;
   decode_ws_layout(num_seqs, num_q_heads, head_dim, splits, &ob, &mb);
   return ob + mb;
@@ -256,13 +295,16 @@ static pa_status decode_impl(void* out, const void* q, int64_t q_token_stride, c
   if (max_blocks_per_seq <= 0) return fail(PA_ERR_INVALID_ARG, "max_blocks_per_seq must be positive");
   if ((int64_t)max_blocks_per_seq * block_size < max_context_len)
     return fail(PA_ERR_INVALID_ARG, "max_blocks_per_seq*block_size < max_context_len");
+  if ((int64_t)num_blocks * block_size < max_context_len)
+    return fail(PA_ERR_INVALID_ARG, "max_context_len exceeds the pool (num_blocks*block_size)");
   if (!(scale > 0.f) || !std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale must be finite and > 0");
   if (partition_size < 0 || partition_size % 64)
     return fail(PA_ERR_INVALID_ARG, "partition_size must be 0 (auto) or a positive multiple of 64");
-  int p = partition_size > 0 ? partition_size
-                             : decode_auto_partition(num_seqs, num_kv_heads, max_context_len);
-  int splits = (max_context_len + p - 1) / p;
-  if (splits > 65535) return fail(PA_ERR_UNSUPPORTED, "too many partitions; raise partition_size");
+  const int p = partition_size > 0 ? partition_size
+                                   : decode_auto_partition(num_seqs, num_kv_heads, max_context_len);
+  const int64_t splits64 = ((int64_t)max_context_len + p - 1) / p;
+  if (splits64 > 65535) return fail(PA_ERR_UNSUPPORTED, "too many partitions; raise partition_size");
+  const int splits = (int)splits64;
   DecodeArgs a{};
   a.out = out; a.q = q; a.q_stride = q_token_stride;
   a.k_cache = k_cache; a.v_cache = v_cache;

@@ -14,9 +14,9 @@
 
 namespace pa {
 
-// Launches `kern` on `stream` with programmatic stream serialization allowed
-// (the kernels call pdl_wait() before reading inputs), unless PA_PDL=0.
-bool pdl_enabled();
+// Launches `kern` on `stream` with programmatic stream serialization allowed:
+// the kernels call pdl_wait() before reading inputs, so a launch may be
+// scheduled while the previous kernel on the stream drains.
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
                               cudaStream_t stream, Args&&... args) {
@@ -29,19 +29,30 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
+
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` on the current
+// device.  The attribute belongs to the device's context, so it is set once
+// per device (and again after a context is re-created: a launch that fails
+// with too little shared memory clears the record).
+pa_status ensure_smem_attr(const void* kernel, int bytes, const char* what);
+void forget_smem_attr(const void* kernel);
+
+// Number of SMs of the current device (cached per device).
+int device_sm_count();
 
 // Records `msg` as this thread's last error and returns `s`.
 pa_status fail(pa_status s, const std::string& msg);
 pa_status cuda_fail(cudaError_t e, const char* what);
 
 // A 3-D view [rows, heads, head_dim] of a bf16 buffer (a KV pool or packed q)
-// as a TMA tensor map with 128-byte swizzle and boxes of {64, 1, box_rows}.
-// Cached per (pointer, shape, box); thread-safe.  Fills *out on success.
+// as a TMA tensor map with 128-byte swizzle and boxes of {64, box_heads,
+// box_rows}.  Cached per (pointer, shape, box); thread-safe.  Fills *out on
+// success.
 pa_status get_tensor_map(CUtensorMap* out, const void* base, int64_t rows, int heads, int head_dim,
-                         int64_t row_stride_elems, int box_rows);
+                         int64_t row_stride_elems, int box_rows, int box_heads = 1);
 
 struct DecodeArgs {
   void* out;

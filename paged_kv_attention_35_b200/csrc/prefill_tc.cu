@@ -1,36 +1,51 @@
 // prefill_tc.cu -- varlen causal prefill over the paged pool on the 5th-gen
-// tensor cores (tcgen05 + TMEM), head_dim 128.
+// tensor cores (tcgen05 + TMEM), head_dim 64 or 128.
 //
-// Definition (same as prefill_mma.cu): sequence i computes q_len new queries
-// over k_len keys, the first k_len - q_len a cached prefix shared through the
-// hash prefix cache ("Prefix Caching via hashing", lnwmold.com item); query j
-// attends keys 0 .. k_len-q_len+j; prompts are batched by cumulative sequence
-// lengths ("Preparation before computation", same item).
+// Definition: sequence i computes q_len new queries over k_len keys, the
+// first k_len - q_len a cached prefix shared through the hash prefix cache
+// ("Prefix Caching via hashing", lnwmold.com item); query j attends keys
+// 0 .. k_len-q_len+j (bottom-right causal); prompts are batched by cumulative
+// sequence lengths ("Preparation before computation", same item).  Query head
+// h reads KV head h / G.
 //
-// One CTA = two consecutive 128-row query tiles (A, B) of one (sequence,
-// query head); 10 warps:
-//   warp 8      TMA producer: both Q tiles once, then 128-key K and V tiles of
-//               the sequence (one box per physical-block chunk, 128-byte
-//               swizzle) into a 5-slot ring (K_j, V_j, K_j+1, ...) shared by
-//               both tiles; zeroes V rows of the last tile past the CTA's last
-//               visible key (stale pool rows may hold NaN).
-//   warp 9      MMA issuer (one thread): S_t(j) = Q_t K_j^T into tile t's TMEM
-//               S buffer (M=128, N=128, K=16 x 8) and O_t += P_t(j) V_j into its
-//               TMEM O accumulator (A = P read from TMEM, B = V MN-major),
-//               interleaving the tiles so one tile's softmax overlaps the other
-//               tile's MMAs; tcgen05.commit signals the mbarriers.
-//   warps 0-3 / 4-7   softmax of tile A / B, one thread per query row (TMEM
-//               lane): tcgen05.ld the S row, causal mask on diagonal tiles only,
-//               online softmax in the log2 domain with a lazy rescale (the
-//               reference max moves only when it grows by more than 8, a factor
-//               256), P as bf16 pairs written back over the S columns it came
-//               from (tcgen05.st), O rescaled in TMEM when needed; epilogue
-//               O / l -> bf16 -> global.
-// TMEM: 512 columns (S_A/P_A | O_A | S_B/P_B | O_B).  The MMA thread issues
-// P V of a tile before that tile's next Q K^T, and tcgen05 MMAs of one thread
-// run in issue order, so the next S never overwrites P before P V has read it.
-// Shared memory: Q 2 x 32 KB, K/V ring 5 x 32 KB.  Every wait is bounded; an
-// abort winds all roles down, drains the issued MMAs and frees TMEM.
+// Tiles.  The G query heads of one KV head share every K/V byte, so an MMA
+// tile packs qpt = floor(128 / G) consecutive queries x the G heads of one KV
+// head as its M rows (row r = query r / G, head r % G; G = 7: 18 queries x 7
+// heads = 126 rows).  One TMA box {64 hdim, G heads, qpt queries} of the packed
+// q lands exactly in that row order.  A tile's keys end at its last query's
+// position, so the causal band wasted inside a tile is qpt keys wide instead
+// of 128.
+//
+// Work unit = two consecutive query tiles (A = the later, B) of one
+// (sequence, KV head), reading the same K/V tiles.  Units are enumerated as
+// (pair from the end of the sequence, sequence, KV head), KV head fastest, so
+// the longest pairs come first and units that share K/V run side by side.
+// The kernel is persistent: one CTA per SM walks units blockIdx.x,
+// blockIdx.x + gridDim.x, ...; the K/V ring streams across unit boundaries and
+// the next unit's Q and first S overlap the current unit's epilogue.
+//
+// Roles (10 warps):
+//   warp 8   producer: Q tiles (one box per head-dim half) into two Q buffers,
+//            then 128-key K and V tiles (one box per physical-block chunk,
+//            128-byte swizzle) into a 5-slot ring; zeroes the V rows past a
+//            unit's last key (stale pool rows may hold NaN).
+//   warp 9   MMA issuer (one thread): S_t(j) = Q_t K_j^T into tile t's TMEM S
+//            buffer (M=128, N=128, K=16 steps); O_t += P_t(j) V_j with P read
+//            from TMEM (TS form, B = V MN-major); tiles A and B interleaved so
+//            one tile's softmax overlaps the other's MMAs.
+//   warps 0-3 / 4-7   softmax of tile A / B, one thread per M row (TMEM lane):
+//            causal mask on the tiles that reach past a row's last key; online
+//            softmax in the log2 domain with a lazy rescale (the reference max
+//            moves only when it grows by more than 8, i.e. 256x); a fixed share
+//            of the exponentials is evaluated on the FMA pipe (exp2_poly2) so
+//            the MUFU unit is not the only one doing them; P as bf16 pairs
+//            written back over the S columns; epilogue O / l -> bf16 -> global.
+// TMEM: 512 columns (S_A/P_A | O_A | S_B/P_B | O_B).  MMAs of one thread run
+// in issue order, so the next S never overwrites P before P V has read it, and
+// a unit's first P V into O_t is issued only after tile t's softmax warps,
+// which also run its epilogue, have read the previous unit's O_t.
+// Every wait is bounded; an abort winds all roles down, drains the issued
+// MMAs and frees TMEM.
 
 #include <cmath>
 
@@ -40,27 +55,73 @@
 
 namespace pa {
 
-constexpr int kTcRows = 128;     // query rows per tile (MMA M)
+constexpr int kTcRows = 128;     // MMA M: packed (query, head) rows of a tile
 constexpr int kTcKeys = 128;     // keys per KV tile (MMA N of QK^T, K of PV)
 constexpr int kTcThreads = 320;  // 2 softmax warpgroups + producer warp + MMA warp
-constexpr int kTile = 32768;     // one 128 x 128 bf16 operand: two 128 x 64 swizzled halves
-constexpr int kHalf = 16384;
+constexpr int kTcHalf = kTcRows * 128;  // one 128-row x 64-element bf16 half (swizzled)
 constexpr int kRing = 5;         // K/V ring slots (K_j, V_j, K_j+1, ... in turn)
 constexpr float kLazyRescale = 8.f;   // log2 of the largest un-rescaled growth (256x)
+
+// Exponentials evaluated by polynomial: pair k of every 8 value pairs (16
+// scores) is emulated when bit k is set.
+constexpr uint32_t kEmuPairs = 0x4A;   // pairs 1, 3, 6: 3 of 8
 
 struct PrefillTcParams {
   __nv_bfloat16* out;
   const int32_t* cu_q;
   const int32_t* cu_k;
   const int32_t* block_tables;
-  int max_blocks;
-  int hq, group;
+  int max_blocks, num_seqs;
+  int hq, hkv, group, qpt, rows;
   int block_size, log2_bs, box_rows;
   int num_blocks, num_slots;
   int max_seqlen_q, max_seqlen_k, total_q;
+  int64_t total_units;             // pairs x sequences x KV heads (some empty)
   float scale_log2;
   int32_t* err_flag;
 };
+
+// One work unit: tiles A (t = 0) and B (t = 1) of a (sequence, KV head).
+struct TcUnit {
+  int kvh, q_start, q_len, k_len, cached;
+  int q0[2];        // first query of tile t within the sequence
+  int nt[2];        // KV tiles tile t reads (nt[1] == 0: no tile B)
+  int kv_end;       // keys tile A reads (tile B reads no more)
+};
+
+// 1: a unit with work, 0: an empty slot, -1: invalid sequence lengths.
+__device__ __forceinline__ int decode_unit(const PrefillTcParams& p, int64_t idx, TcUnit& u) {
+  const int kvh = (int)(idx % p.hkv);
+  const int64_t r = idx / p.hkv;
+  const int seq = (int)(r % p.num_seqs);
+  const int pp = (int)(r / p.num_seqs);
+  const int cq0 = __ldg(p.cu_q + seq), cq1 = __ldg(p.cu_q + seq + 1);
+  const int ck0 = __ldg(p.cu_k + seq), ck1 = __ldg(p.cu_k + seq + 1);
+  const int q_len = cq1 - cq0, k_len = ck1 - ck0;
+  if (!(cq0 >= 0 && q_len >= 0 && cq1 <= p.total_q && k_len >= q_len &&
+        q_len <= p.max_seqlen_q && k_len <= p.max_seqlen_k && k_len <= p.max_blocks * p.block_size))
+    return pp == 0 && kvh == 0 ? -1 : 0;
+  const int T = (q_len + p.qpt - 1) / p.qpt;
+  if (2 * pp >= T) return 0;
+  u.kvh = kvh;
+  u.q_start = cq0;
+  u.q_len = q_len;
+  u.k_len = k_len;
+  u.cached = k_len - q_len;
+  const int ta = T - 1 - 2 * pp, tb = ta - 1;
+  u.q0[0] = ta * p.qpt;
+  u.kv_end = min(k_len, u.cached + min(q_len, u.q0[0] + p.qpt));
+  u.nt[0] = (u.kv_end + kTcKeys - 1) / kTcKeys;
+  if (tb >= 0) {
+    u.q0[1] = tb * p.qpt;
+    const int e = min(k_len, u.cached + min(q_len, u.q0[1] + p.qpt));
+    u.nt[1] = (e + kTcKeys - 1) / kTcKeys;
+  } else {
+    u.q0[1] = 0;
+    u.nt[1] = 0;
+  }
+  return 1;
+}
 
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                         int32_t* err_flag) {
@@ -100,35 +161,65 @@ __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
 }
 __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   uint64_t d;
-  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
 
-constexpr int kBtCache = 256;    // block-table entries staged in shared memory
+// 2^x for two values on the FMA pipe.  x is clamped to >= -125 (2^-125 is
+// below anything that survives the bf16 rounding of P next to a 1), then
+// split as x = j + f with j the nearest integer (adding and subtracting
+// 1.5 * 2^23 rounds to an integer in the low mantissa bits) and f in
+// [-0.5, 0.5]; 2^f is a cubic whose coefficients were fitted to minimise the
+// relative error on that interval (iteratively reweighted least squares; max
+// relative error 7.5e-5, against 2^-9 for the bf16 rounding of P), and j is
+// added to the exponent field.
+struct Exp2Poly {
+  uint64_t magic, neg_magic, neg_one, c3, c2, c1, c0;
+  __device__ __forceinline__ Exp2Poly() {
+    magic = f32x2(12582912.f, 12582912.f);
+    neg_magic = f32x2(-12582912.f, -12582912.f);
+    neg_one = f32x2(-1.f, -1.f);
+    c3 = f32x2(0.0551706925f, 0.0551706925f);
+    c2 = f32x2(0.2426096499f, 0.2426096499f);
+    c1 = f32x2(0.6932610273f, 0.6932610273f);
+    c0 = f32x2(0.9999281764f, 0.9999281764f);
+  }
+  __device__ __forceinline__ void eval(float x0, float x1, float& e0, float& e1) const {
+    const uint64_t x = f32x2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+    const uint64_t t = fadd2(x, magic);              // j + 1.5 * 2^23
+    const uint64_t f = ffma2(fadd2(t, neg_magic), neg_one, x);   // x - j
+    uint64_t q = ffma2(f, c3, c2);
+    q = ffma2(q, f, c1);
+    q = ffma2(q, f, c0);
+    float q0, q1, t0, t1;
+    f32x2_split(q, q0, q1);
+    f32x2_split(t, t0, t1);
+    e0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+    e1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+  }
+};
 
-// Barrier block in shared memory (after the operand buffers).
 struct TcBars {
-  uint64_t q_full;
+  uint64_t q_full[2];      // Q tile t landed
+  uint64_t q_empty[2];     // the last Q_t K^T of a unit is complete: Q buffer t free
   uint64_t kv_full[kRing];
   uint64_t kv_empty[kRing];
+  uint64_t vz[kRing];      // a unit's last V tile landed in this slot and its tail is zeroed
   uint64_t s_full[2];      // per query tile (A, B)
   uint64_t p_full[2];
   uint64_t pv_done[2];
-  uint64_t vz_ready;
   uint64_t drain;
   uint32_t tmem;
   int abort_flag;
-  int bt[kBtCache];        // the sequence's first block-table entries
 };
 
-// One CTA = two consecutive 128-row query tiles (A, B) of one (sequence, head).
-// The MMA thread interleaves them so that the softmax of one tile overlaps the
-// other tile's P V and next Q K^T on the tensor core:
-//   S_A(0) S_B(0) | PV_A(0) S_A(1) | PV_B(0) S_B(1) | PV_A(1) S_A(2) | ...
-// Both tiles read the same K/V tiles (the later tile needs at most one more).
+template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const PrefillTcParams p) {
+  constexpr int kHalves = D / 64;
+  constexpr int kTile = kHalves * kTcHalf;     // one Q, K or V tile
+  constexpr int kSteps = D / 16;               // K steps of Q K^T
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -137,72 +228,42 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   TcBars* bar = reinterpret_cast<TcBars*>(sKV + kRing * kTile);
   volatile int* abort_flag = &bar->abort_flag;
 
-  // pair 0 = the sequence's last two query tiles (they see the most keys), so
-  // launch order is longest first and every CTA but possibly a sequence's
-  // first carries two tiles; tile A is the later one of the pair.
   pdl_wait();
   pdl_trigger();
-  const int pp = blockIdx.x;
-  const int h = blockIdx.y, seq = blockIdx.z;
-  const int kvh = h / p.group;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const int cq0 = __ldg(p.cu_q + seq), cq1 = __ldg(p.cu_q + seq + 1);
-  const int ck0 = __ldg(p.cu_k + seq), ck1 = __ldg(p.cu_k + seq + 1);
-  const int q_start = cq0, q_len = cq1 - cq0, k_len = ck1 - ck0;
-  if (!(cq0 >= 0 && q_len >= 0 && cq1 <= p.total_q && k_len >= q_len &&
-        q_len <= p.max_seqlen_q && k_len <= p.max_seqlen_k && k_len <= p.max_blocks * p.block_size)) {
-    if (threadIdx.x == 0 && blockIdx.x == 0 && h == 0) raise_flag(p.err_flag, PA_FLAG_LEN_OOB);
-    return;
-  }
-  const int T = (q_len + kTcRows - 1) / kTcRows;   // query tiles of the sequence
-  if (2 * pp >= T) return;
-  const int tile_a = T - 1 - 2 * pp, tile_b = tile_a - 1;
-  const bool hasB = tile_b >= 0;
-  const int q0A = tile_a * kTcRows;
-  const int q0B = hasB ? tile_b * kTcRows : 0;
-  const int cached = k_len - q_len;
-  const int kv_endA = min(k_len, cached + min(q_len, q0A + kTcRows));
-  const int kv_endB = hasB ? min(k_len, cached + min(q_len, q0B + kTcRows)) : 0;
-  const int nA = (kv_endA + kTcKeys - 1) / kTcKeys;
-  const int nB = (kv_endB + kTcKeys - 1) / kTcKeys;
-  const int kv_end = max(kv_endA, kv_endB);
-  const int n = max(nA, nB);
-  const int last_valid = kv_end - (n - 1) * kTcKeys;
-  const bool zero_tail = last_valid < kTcKeys;
-  const int32_t* bt = p.block_tables + (int64_t)seq * p.max_blocks;
-
   if (warp == 8 && lane == 0) {
-    // the producer thread sets up the barriers and starts the Q loads at once
-    mbar_init(&bar->q_full, 1);
+    mbar_init(&bar->q_full[0], 1);
+    mbar_init(&bar->q_full[1], 1);
+    mbar_init(&bar->q_empty[0], 1);
+    mbar_init(&bar->q_empty[1], 1);
     for (int s = 0; s < kRing; ++s) {
       mbar_init(&bar->kv_full[s], 1);
       mbar_init(&bar->kv_empty[s], 1);
+      mbar_init(&bar->vz[s], 1);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bar->s_full[t], 1);
       mbar_init(&bar->p_full[t], 4);
       mbar_init(&bar->pv_done[t], 1);
     }
-    mbar_init(&bar->vz_ready, 1);
     mbar_init(&bar->drain, 1);
     bar->abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
-    mbar_arrive_expect_tx(&bar->q_full, hasB ? 2 * kTile : kTile);
-    tma_load_3d(sQ, &tmQ, &bar->q_full, 0, h, q_start + q0A);
-    tma_load_3d(sQ + kHalf, &tmQ, &bar->q_full, 64, h, q_start + q0A);
-    if (hasB) {
-      tma_load_3d(sQ + kTile, &tmQ, &bar->q_full, 0, h, q_start + q0B);
-      tma_load_3d(sQ + kTile + kHalf, &tmQ, &bar->q_full, 64, h, q_start + q0B);
-    }
   }
-  if (warp == 8) {
-    // stage the block-table entries this CTA reads (all lanes, one round trip)
-    const int nblk = min((kv_end + p.block_size - 1) >> p.log2_bs, kBtCache);
-    for (int i = lane; i < nblk; i += 32) bar->bt[i] = __ldg(bt + i);
+  // rows >= p.rows of the Q buffers are never written by TMA: zero them once so
+  // the padding rows of S stay finite
+  {
+    const int pad = kTcRows - p.rows;
+    for (int i = threadIdx.x; i < 2 * kHalves * pad * 8; i += kTcThreads) {
+      const int chunk = i & 7, rr = (i >> 3) % pad, hb = (i >> 3) / pad;   // hb = buffer * kHalves + half
+      *reinterpret_cast<uint4*>(sQ + hb * kTcHalf + (p.rows + rr) * 128 + chunk * 16) =
+          make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
   }
   if (warp == 9) {
     tc::tmem_alloc(&bar->tmem, 512);
@@ -211,125 +272,170 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  // tile t: S at TMEM columns [256t, 256t+128) with P (bf16 pairs) over its first
-  // 64 columns once S has been read; O at [256t+128, 256t+256)
+  // tile t: S at TMEM columns [256t, 256t+128) with P (bf16 pairs) over its
+  // first 64 columns once S has been read; O at [256t+128, 256t+128+D)
   const uint32_t tmem = bar->tmem;
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      const int box = p.box_rows;
-      int i = 0;
-      for (int j = 0; j < n; ++j) {
-        const int t0 = j * kTcKeys;
-        const int nbox = (min(kTcKeys, kv_end - t0) + box - 1) / box;
-        const uint32_t bytes = (uint32_t)(nbox * box * 128 * 2);
-        int rows[kTcKeys / 16];
-        for (int b = 0; b < nbox; ++b) {
-          const int t = t0 + b * box;
-          const int lb = t >> p.log2_bs;
-          const int bid = lb < kBtCache ? bar->bt[lb] : __ldg(bt + lb);
-          if (bid < 0 || bid >= p.num_blocks) {
-            raise_flag(p.err_flag, PA_FLAG_BLOCK_OOB);
-            rows[b] = p.num_slots;                 // past the pool: TMA fills zeros
-          } else {
-            rows[b] = bid * p.block_size + (t & (p.block_size - 1));
-          }
-        }
-        bool ok = true;
-        for (int kv = 0; kv < 2; ++kv, ++i) {
-          const int slot = i % kRing;
-          if (i >= kRing &&
-              !tc_wait(&bar->kv_empty[slot], ((i / kRing) - 1) & 1, abort_flag, p.err_flag)) {
+    uint32_t kv_i = 0, qn[2] = {0, 0}, vz_bits = 0;
+    const int box = p.box_rows;
+    for (int64_t ui = blockIdx.x; ui < p.total_units; ui += gridDim.x) {
+      TcUnit u;
+      const int st = decode_unit(p, ui, u);
+      if (st < 0 && lane == 0) raise_flag(p.err_flag, PA_FLAG_LEN_OOB);
+      if (st <= 0) continue;
+      const int n = u.nt[0];
+      const int32_t* bt = p.block_tables + (int64_t)(ui / p.hkv % p.num_seqs) * p.max_blocks;
+      bool ok = true;
+      if (lane == 0) {
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (u.nt[t] == 0) continue;
+          if (qn[t] > 0 && !tc_wait(&bar->q_empty[t], (qn[t] - 1) & 1, abort_flag, p.err_flag)) {
             ok = false;
             break;
           }
-          const CUtensorMap* map = kv ? &tmV : &tmK;
-          mbar_arrive_expect_tx(&bar->kv_full[slot], bytes);
+          mbar_arrive_expect_tx(&bar->q_full[t], (uint32_t)(kHalves * p.rows * 128));
+#pragma unroll
+          for (int hf = 0; hf < kHalves; ++hf)
+            tma_load_3d(sQ + t * kTile + hf * kTcHalf, &tmQ, &bar->q_full[t], hf * 64,
+                        u.kvh * p.group, u.q_start + u.q0[t]);
+          ++qn[t];
+        }
+        for (int j = 0; j < n && ok; ++j) {
+          const int t0 = j * kTcKeys;
+          const int nbox = (min(kTcKeys, u.kv_end - t0) + box - 1) / box;
+          const uint32_t bytes = (uint32_t)(nbox * box * 128 * kHalves);
+          int rows[kTcKeys / 16];
           for (int b = 0; b < nbox; ++b) {
-            uint8_t* dst = sKV + slot * kTile + b * box * 128;
-            tma_load_3d(dst, map, &bar->kv_full[slot], 0, kvh, rows[b]);
-            tma_load_3d(dst + kHalf, map, &bar->kv_full[slot], 64, kvh, rows[b]);
+            const int t = t0 + b * box;
+            const int bid = __ldg(bt + (t >> p.log2_bs));
+            if (bid < 0 || bid >= p.num_blocks) {
+              raise_flag(p.err_flag, PA_FLAG_BLOCK_OOB);
+              rows[b] = p.num_slots;                 // past the pool: TMA fills zeros
+            } else {
+              rows[b] = bid * p.block_size + (t & (p.block_size - 1));
+            }
+          }
+          for (int kv = 0; kv < 2; ++kv, ++kv_i) {
+            const int slot = kv_i % kRing;
+            if (kv_i >= kRing &&
+                !tc_wait(&bar->kv_empty[slot], ((kv_i / kRing) - 1) & 1, abort_flag, p.err_flag)) {
+              ok = false;
+              break;
+            }
+            const CUtensorMap* map = kv ? &tmV : &tmK;
+            mbar_arrive_expect_tx(&bar->kv_full[slot], bytes);
+            for (int b = 0; b < nbox; ++b) {
+              uint8_t* dst = sKV + slot * kTile + b * box * 128;
+#pragma unroll
+              for (int hf = 0; hf < kHalves; ++hf)
+                tma_load_3d(dst + hf * kTcHalf, map, &bar->kv_full[slot], hf * 64, u.kvh, rows[b]);
+            }
           }
         }
-        if (!ok) break;
       }
-    }
-    __syncwarp();
-    if (zero_tail) {
-      const int iv = 2 * (n - 1) + 1, slot = iv % kRing;
-      if (tc_wait(&bar->kv_full[slot], (iv / kRing) & 1, abort_flag, p.err_flag)) {
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (lane != 0) kv_i += 2 * n;                 // lane 0 counted its loads above
+      if (!ok) break;
+      // zero the last V tile's rows past the unit's last key
+      const int last_valid = u.kv_end - (n - 1) * kTcKeys;
+      if (last_valid < kTcKeys) {
+        const uint32_t iv = kv_i - 1, slot = iv % kRing;
+        bool landed = true;
+        if (lane == 0) landed = tc_wait(&bar->kv_full[slot], (iv / kRing) & 1, abort_flag, p.err_flag);
+        if (!__shfl_sync(0xffffffffu, landed ? 1 : 0, 0)) break;
         const int nrow = kTcKeys - last_valid;
-        for (int t = lane; t < nrow * 16; t += 32) {
-          const int hf = t / (nrow * 8);
-          const int rr = (t / 8) % nrow;
-          *reinterpret_cast<uint4*>(sKV + slot * kTile + hf * kHalf + (last_valid + rr) * 128 +
-                                    (t & 7) * 16) = make_uint4(0, 0, 0, 0);
+        for (int i = lane; i < nrow * 8 * kHalves; i += 32) {
+          const int hf = i / (nrow * 8);
+          const int rr = (i >> 3) % nrow;
+          *reinterpret_cast<uint4*>(sKV + slot * kTile + hf * kTcHalf + (last_valid + rr) * 128 +
+                                    (i & 7) * 16) = make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->vz[slot]);
+        vz_bits ^= 1u << slot;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar->vz_ready);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = tc::idesc_bf16(kTcRows, kTcKeys, false, false);
-      constexpr uint32_t idO = tc::idesc_bf16(kTcRows, 128, false, true);
-      const int ntile[2] = {nA, nB};
+      constexpr uint32_t idO = tc::idesc_bf16(kTcRows, D, false, true);
       // descriptors are built once; stepping K adds (byte offset / 16) to the
       // start-address field (no carry: shared addresses stay below 256 KB)
       const uint64_t dQ0 = tc::sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t dK0 = tc::sdesc_sw128(smem_u32(sKV), 16, 1024);
-      const uint64_t dV0 = tc::sdesc_sw128(smem_u32(sKV), kHalf, 1024);
-      auto issue_s = [&](int t, int j) {          // S_t(j) = Q_t K_j^T
-        const int slot = (2 * j) % kRing;
+      const uint64_t dV0 = tc::sdesc_sw128(smem_u32(sKV), kTcHalf, 1024);
+      uint32_t kv_i = 0, qc[2] = {0, 0}, pc[2] = {0, 0}, vz_bits = 0;
+      bool ok = true;
+      auto wait_kv = [&](uint32_t i) {
+        return tc_wait(&bar->kv_full[i % kRing], (i / kRing) & 1, abort_flag, p.err_flag);
+      };
+      auto issue_s = [&](int t, uint32_t kslot) {          // S_t = Q_t K^T
         const uint64_t dQ = dQ0 + (uint64_t)((t * kTile) >> 4);
-        const uint64_t dK = dK0 + (uint64_t)((slot * kTile) >> 4);
+        const uint64_t dK = dK0 + (uint64_t)((kslot * kTile) >> 4);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t o = (uint64_t)(((ks >> 2) * kHalf + (ks & 3) * 32) >> 4);
+        for (int ks = 0; ks < kSteps; ++ks) {
+          const uint64_t o = (uint64_t)(((ks >> 2) * kTcHalf + (ks & 3) * 32) >> 4);
           tc::mma_ss(tmem + 256 * t, dQ + o, dK + o, idS, ks > 0);
         }
         tc::commit(&bar->s_full[t]);
       };
-      auto wait_k = [&](int j) {
-        const int i = 2 * j;
-        return tc_wait(&bar->kv_full[i % kRing], (i / kRing) & 1, abort_flag, p.err_flag);
-      };
-      bool ok = tc_wait(&bar->q_full, 0, abort_flag, p.err_flag) && wait_k(0);
-      if (ok) {
+      for (int64_t ui = blockIdx.x; ok && ui < p.total_units; ui += gridDim.x) {
+        TcUnit u;
+        if (decode_unit(p, ui, u) <= 0) continue;
+        const int n = u.nt[0];
+        for (int t = 0; t < 2 && ok; ++t)
+          if (u.nt[t] > 0) ok = tc_wait(&bar->q_full[t], qc[t]++ & 1, abort_flag, p.err_flag);
+        if (!ok || !wait_kv(kv_i)) break;
         tc::fence_after_sync();
-        issue_s(0, 0);
-        if (nB > 0) issue_s(1, 0);
-        tc::commit(&bar->kv_empty[0]);          // K_0 consumed by both tiles
-      }
-      for (int j = 0; ok && j < n; ++j) {
-        const int iv = 2 * j + 1, vslot = iv % kRing;
-        const bool vz = zero_tail && j == n - 1;
-        // operands first (normally resident long before the softmax is done), so
-        // nothing but the P handshake sits between consecutive MMA groups
-        if (!tc_wait(vz ? &bar->vz_ready : &bar->kv_full[vslot], vz ? 0u : (uint32_t)((iv / kRing) & 1),
-                     abort_flag, p.err_flag) ||
-            (j + 1 < n && !wait_k(j + 1))) {
-          ok = false;
-          break;
-        }
         for (int t = 0; t < 2; ++t) {
-          if (j >= ntile[t]) continue;
-          if (!tc_wait(&bar->p_full[t], j & 1, abort_flag, p.err_flag)) { ok = false; break; }
-          tc::fence_after_sync();
-          const uint64_t dV = dV0 + (uint64_t)((vslot * kTile) >> 4);
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            tc::mma_ts(tmem + 256 * t + 128, tmem + 256 * t + ks * 8,
-                       dV + (uint64_t)((ks * 2048) >> 4), idO, (j > 0 || ks > 0));
-          if (j == ntile[t] - 1) tc::commit(&bar->pv_done[t]);   // the epilogue waits on it
-          if (j + 1 < ntile[t]) issue_s(t, j + 1);
+          if (u.nt[t] == 0) continue;
+          issue_s(t, kv_i % kRing);
+          if (u.nt[t] == 1) tc::commit(&bar->q_empty[t]);
         }
-        if (!ok) break;
-        tc::commit(&bar->kv_empty[vslot]);                 // V_j consumed
-        if (j + 1 < n) tc::commit(&bar->kv_empty[(2 * (j + 1)) % kRing]);   // K_j+1 consumed
+        tc::commit(&bar->kv_empty[kv_i % kRing]);          // K_0 consumed
+        const bool zero_tail = u.kv_end - (n - 1) * kTcKeys < kTcKeys;
+        for (int j = 0; ok && j < n; ++j) {
+          const uint32_t iv = kv_i + 2 * j + 1, vslot = iv % kRing;
+          const uint32_t kn = iv + 1, kslot = kn % kRing;  // K_j+1
+          // operands first (normally resident long before the softmax is done)
+          bool got;
+          if (zero_tail && j == n - 1) {
+            got = tc_wait(&bar->vz[vslot], (vz_bits >> vslot) & 1, abort_flag, p.err_flag);
+            vz_bits ^= 1u << vslot;
+          } else {
+            got = wait_kv(iv);
+          }
+          if (!got || (j + 1 < n && !wait_kv(kn))) {
+            ok = false;
+            break;
+          }
+          for (int t = 0; t < 2; ++t) {
+            if (j >= u.nt[t]) continue;
+            if (!tc_wait(&bar->p_full[t], pc[t]++ & 1, abort_flag, p.err_flag)) {
+              ok = false;
+              break;
+            }
+            tc::fence_after_sync();
+            const uint64_t dV = dV0 + (uint64_t)((vslot * kTile) >> 4);
+#pragma unroll
+            for (int ks = 0; ks < kTcKeys / 16; ++ks)
+              tc::mma_ts(tmem + 256 * t + 128, tmem + 256 * t + ks * 8,
+                         dV + (uint64_t)((ks * 2048) >> 4), idO, (j > 0 || ks > 0));
+            if (j == u.nt[t] - 1) tc::commit(&bar->pv_done[t]);   // the epilogue waits on it
+            if (j + 1 < u.nt[t]) {
+              issue_s(t, kslot);
+              if (j + 2 == u.nt[t]) tc::commit(&bar->q_empty[t]);
+            }
+          }
+          if (!ok) break;
+          tc::commit(&bar->kv_empty[vslot]);                 // V_j consumed
+          if (j + 1 < n) tc::commit(&bar->kv_empty[kslot]);  // K_j+1 consumed
+        }
+        kv_i += 2 * n;
       }
       // every issued MMA finishes before TMEM is released
       tc::commit(&bar->drain);
@@ -338,93 +444,112 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax (warpgroup t = tile)
     const int t = warp >> 2;                       // 0: tile A, 1: tile B
-    const int r = threadIdx.x & 127;               // row within the tile = TMEM lane
-    const int nt = t ? nB : nA;
-    const int q0 = t ? q0B : q0A;
+    const int r = threadIdx.x & 127;               // M row = TMEM lane
+    const int qi = r / p.group, hh = r - qi * p.group;   // query within the tile, head in the group
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + 256 * t + lane_off, tO = tS + 128;
-    const int limit = min(cached + q0 + r, k_len - 1);   // last visible key of this row
     const float sl2 = p.scale_log2;
-    float m_ref = -INFINITY, l = 0.f;
+    const Exp2Poly ex;
+    uint32_t sc = 0, pvc = 0;
     bool ok = true;
-    float sv[kTcKeys];
-    for (int j = 0; j < nt; ++j) {
-      // S_t(j) complete implies every earlier MMA of this CTA -- P V of tile j-1
-      // included -- is complete: O may be rescaled and the S/P columns reused.
-      if (!tc_wait(&bar->s_full[t], j & 1, abort_flag, p.err_flag)) { ok = false; break; }
-      tc::fence_after_sync();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tc::ld32(tS + c * 32, reinterpret_cast<uint32_t*>(sv) + c * 32);
-      tc::wait_ld();
-      const int t0 = j * kTcKeys;
-      if (t0 + kTcKeys - 1 > limit) {              // diagonal / tail tile: mask
-        const int lim = limit - t0;
-#pragma unroll
-        for (int i = 0; i < kTcKeys; ++i) sv[i] = i <= lim ? sv[i] : -INFINITY;
-      }
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int i = 0; i < kTcKeys; i += 8) {
-        mx4[0] = max3f(mx4[0], sv[i + 0], sv[i + 1]);
-        mx4[1] = max3f(mx4[1], sv[i + 2], sv[i + 3]);
-        mx4[2] = max3f(mx4[2], sv[i + 4], sv[i + 5]);
-        mx4[3] = max3f(mx4[3], sv[i + 6], sv[i + 7]);
-      }
-      const float mx = max3f(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * sl2;  // scale > 0
-      float alpha = 1.f;
-      bool resc = false;
-      if (m_ref == -INFINITY) {
-        m_ref = mx;
-      } else if (mx > m_ref + kLazyRescale) {
-        alpha = fast_exp2(m_ref - mx);
-        m_ref = mx;
-        resc = true;
-        l *= alpha;
-      }
-      const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
-      const uint64_t sc2 = f32x2(sl2, sl2), nm2 = f32x2(neg_m, neg_m);
-      uint64_t rs2[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
-      uint32_t pk[kTcKeys / 2];
-#pragma unroll
-      for (int i = 0; i < kTcKeys; i += 2) {
-        float x0, x1;
-        f32x2_split(ffma2(f32x2(sv[i], sv[i + 1]), sc2, nm2), x0, x1);
-        const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
-        rs2[(i >> 1) & 1] = fadd2(rs2[(i >> 1) & 1], f32x2(e0, e1));
-        pk[i >> 1] = pack_bf16(e0, e1);
-      }
-      {
-        float a0, a1, b0, b1;
-        f32x2_split(rs2[0], a0, a1);
-        f32x2_split(rs2[1], b0, b1);
-        l += (a0 + a1) + (b0 + b1);
-      }
-      tc::st32(tS, pk);                            // P over the first 64 S columns
-      tc::st32(tS + 32, pk + 32);
-      if (__any_sync(0xffffffffu, resc)) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t ov[32];
-          tc::ld32(tO + c * 32, ov);
-          tc::wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-          tc::st32(tO + c * 32, ov);
+    for (int64_t ui = blockIdx.x; ok && ui < p.total_units; ui += gridDim.x) {
+      TcUnit u;
+      if (decode_unit(p, ui, u) <= 0 || u.nt[t] == 0) continue;
+      const int nt = u.nt[t], q0 = u.q0[t];
+      const int limit = min(u.cached + q0 + qi, u.k_len - 1);   // last visible key of this row
+      float m_ref = -INFINITY, l = 0.f;
+      for (int j = 0; j < nt; ++j) {
+        // S_t(j) complete implies every earlier MMA of this CTA -- P V of tile j-1
+        // included -- is complete: O may be rescaled and the S/P columns reused.
+        if (!__all_sync(0xffffffffu, tc_wait(&bar->s_full[t], sc++ & 1, abort_flag, p.err_flag))) {
+          ok = false;
+          break;
         }
+        tc::fence_after_sync();
+        float sv[kTcKeys];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tc::ld32(tS + c * 32, reinterpret_cast<uint32_t*>(sv) + c * 32);
+        tc::wait_ld();
+        const int t0 = j * kTcKeys;
+        if (t0 + kTcKeys - 1 > limit) {            // tile reaches past the row's last key: mask
+          const int lim = limit - t0;
+#pragma unroll
+          for (int i = 0; i < kTcKeys; ++i) sv[i] = i <= lim ? sv[i] : -INFINITY;
+        }
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int i = 0; i < kTcKeys; i += 8) {
+          mx4[0] = max3f(mx4[0], sv[i + 0], sv[i + 1]);
+          mx4[1] = max3f(mx4[1], sv[i + 2], sv[i + 3]);
+          mx4[2] = max3f(mx4[2], sv[i + 4], sv[i + 5]);
+          mx4[3] = max3f(mx4[3], sv[i + 6], sv[i + 7]);
+        }
+        const float mx = max3f(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * sl2;  // scale > 0
+        float alpha = 1.f;
+        bool resc = false;
+        if (m_ref == -INFINITY) {
+          m_ref = mx;
+        } else if (mx > m_ref + kLazyRescale) {
+          alpha = fast_exp2(m_ref - mx);
+          m_ref = mx;
+          resc = true;
+          l *= alpha;
+        }
+        const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
+        const uint64_t sc2 = f32x2(sl2, sl2), nm2 = f32x2(neg_m, neg_m);
+        uint64_t rs2[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
+        // P in two halves of 64 keys, each stored as 32 bf16 pairs over the S
+        // columns it came from (S is already in registers)
+#pragma unroll
+        for (int hk = 0; hk < 2; ++hk) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 64 * hk; i < 64 * hk + 64; i += 2) {
+            float x0, x1, e0, e1;
+            f32x2_split(ffma2(f32x2(sv[i], sv[i + 1]), sc2, nm2), x0, x1);
+            if ((kEmuPairs >> ((i >> 1) & 7)) & 1) {
+              ex.eval(x0, x1, e0, e1);
+            } else {
+              e0 = fast_exp2(x0);
+              e1 = fast_exp2(x1);
+            }
+            rs2[(i >> 1) & 1] = fadd2(rs2[(i >> 1) & 1], f32x2(e0, e1));
+            pk[(i >> 1) & 31] = pack_bf16(e0, e1);
+          }
+          tc::st32(tS + 32 * hk, pk);
+        }
+        {
+          float a0, a1, b0, b1;
+          f32x2_split(rs2[0], a0, a1);
+          f32x2_split(rs2[1], b0, b1);
+          l += (a0 + a1) + (b0 + b1);
+        }
+        if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tc::ld32(tO + c * 32, ov);
+            tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            tc::st32(tO + c * 32, ov);
+          }
+        }
+        tc::wait_st();
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->p_full[t]);
       }
-      tc::wait_st();
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar->p_full[t]);
-    }
-    // epilogue: O / l -> bf16
-    if (nt > 0 && ok && tc_wait(&bar->pv_done[t], 0, abort_flag, p.err_flag)) {
+      if (!ok) break;
+      // epilogue: O / l -> bf16
+      if (!__all_sync(0xffffffffu, tc_wait(&bar->pv_done[t], pvc++ & 1, abort_flag, p.err_flag))) break;
       tc::fence_after_sync();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      const bool store = q0 + r < q_len;
-      __nv_bfloat16* orow = p.out + ((int64_t)(q_start + q0 + r) * p.hq + h) * 128;
+      const bool store = r < p.rows && q0 + qi < u.q_len;
+      __nv_bfloat16* orow =
+          p.out + ((int64_t)(u.q_start + q0 + qi) * p.hq + u.kvh * p.group + hh) * D;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
         tc::ld32(tO + c * 32, ov);
         tc::wait_ld();
@@ -440,6 +565,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
       }
+      // the next unit's first P V overwrites O_t: every lane's reads are done
+      tc::fence_before_sync();
+      __syncwarp();
     }
   }
 
@@ -451,11 +579,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
-pa_status launch_prefill_tc(const PrefillArgs& a) {
+template <int D>
+static pa_status launch_prefill_d(const PrefillArgs& a) {
+  constexpr int kTile = (D / 64) * kTcHalf;
+  const int group = a.hq / a.hkv;
+  if (group > kTcRows) return fail(PA_ERR_UNSUPPORTED, "prefill: more than 128 query heads per KV head");
+  const int qpt = kTcRows / group;
   const int box = a.block_size < kTcKeys ? a.block_size : kTcKeys;
   const int64_t slots = (int64_t)a.num_blocks * a.block_size;
   CUtensorMap mq, mk, mv;
-  pa_status s = get_tensor_map(&mq, a.q, a.total_q, a.hq, a.d, a.q_stride, kTcRows);
+  pa_status s = get_tensor_map(&mq, a.q, a.total_q, a.hq, a.d, a.q_stride, qpt, group);
   if (s != PA_OK) return s;
   s = get_tensor_map(&mk, a.k_cache, slots, a.hkv, a.d, (int64_t)a.hkv * a.d, box);
   if (s != PA_OK) return s;
@@ -467,8 +600,12 @@ pa_status launch_prefill_tc(const PrefillArgs& a) {
   prm.cu_k = a.cu_k;
   prm.block_tables = a.block_tables;
   prm.max_blocks = a.max_blocks;
+  prm.num_seqs = a.num_seqs;
   prm.hq = a.hq;
-  prm.group = a.hq / a.hkv;
+  prm.hkv = a.hkv;
+  prm.group = group;
+  prm.qpt = qpt;
+  prm.rows = qpt * group;
   prm.block_size = a.block_size;
   prm.log2_bs = __builtin_ctz((unsigned)a.block_size);
   prm.box_rows = box;
@@ -477,22 +614,29 @@ pa_status launch_prefill_tc(const PrefillArgs& a) {
   prm.max_seqlen_q = a.max_seqlen_q;
   prm.max_seqlen_k = a.max_seqlen_k;
   prm.total_q = a.total_q;
+  const int64_t max_pairs = ((int64_t)(a.max_seqlen_q + qpt - 1) / qpt + 1) / 2;
+  prm.total_units = max_pairs * a.num_seqs * a.hkv;
   prm.scale_log2 = a.scale * 1.4426950408889634f;
   prm.err_flag = a.err_flag;
-  const size_t smem = (2 + kRing) * (size_t)kTile + 1024 + sizeof(TcBars);
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return cuda_fail(e, "prefill_tc smem attribute");
-    attr_done = true;
+  // at least 120 KB so that two CTAs never share an SM (each allocates all 512
+  // TMEM columns)
+  size_t smem = (2 + kRing) * (size_t)kTile + 1024 + sizeof(TcBars);
+  if (smem < 120 * 1024) smem = 120 * 1024;
+  s = ensure_smem_attr((const void*)prefill_tc_kernel<D>, (int)smem, "prefill smem attribute");
+  if (s != PA_OK) return s;
+  const int64_t ctas = prm.total_units < device_sm_count() ? prm.total_units : device_sm_count();
+  cudaError_t e = launch_pdl(prefill_tc_kernel<D>, dim3((unsigned)ctas), dim3(kTcThreads), smem,
+                             a.stream, mq, mk, mv, prm);
+  if (e != cudaSuccess) {
+    forget_smem_attr((const void*)prefill_tc_kernel<D>);
+    return cuda_fail(e, "prefill launch");
   }
-  if (a.hq > 65535) return fail(PA_ERR_UNSUPPORTED, "too many heads");
-  dim3 grid((a.max_seqlen_q + 2 * kTcRows - 1) / (2 * kTcRows), a.hq, a.num_seqs);
-  cudaError_t e = launch_pdl(prefill_tc_kernel, grid, dim3(kTcThreads), smem, a.stream, mq, mk, mv,
-                             prm);
-  if (e != cudaSuccess) return cuda_fail(e, "prefill_tc launch");
   return PA_OK;
+}
+
+pa_status launch_prefill(const PrefillArgs& a) {
+  if (a.d == 128) return launch_prefill_d<128>(a);
+  return launch_prefill_d<64>(a);
 }
 
 }  // namespace pa

@@ -24,6 +24,16 @@ rows: slot -1, context length 0, which the kernels skip / answer with zeros).
 On the first step of a key the layers run eagerly and the graph is captured
 for the next ones.  Prefill steps always run eagerly.
 
+Timing: ``run`` reports the wall time of the loop, the host time spent inside
+the steps (scheduling, preparation, packing, launching, postprocessing), and
+the GPU time of the steps: for each step the device time from its metadata
+copy to its last kernel, summed (idle device time between steps, while the
+host prepares the next one, is not counted).
+
+``scheduler="priority"`` replays the trace through ``PriorityScheduler``
+(each request gets a seeded priority in ``[0, num_priorities)``; waiting
+sequences are admitted highest priority first).
+
 ``slot_writer`` records, for every pool slot, which (step, packed row) last
 wrote it -- the same for every layer, since all layers share the block tables.
 With the CPU copy of the ring this lets a checker rebuild exactly what any
@@ -40,7 +50,8 @@ import numpy as np
 import torch
 
 from . import synth
-from .host import (Scheduler, SchedulerConfig, Sequence, prepare_decode, prepare_prefill)
+from .host import (PriorityScheduler, Scheduler, SchedulerConfig, Sequence, prepare_decode,
+                   prepare_prefill)
 
 
 @dataclass
@@ -61,6 +72,8 @@ class ReplayConfig:
     max_model_len: int = 4096
     ring: int = 8
     seed: int = synth.SEED_BASE + 5
+    scheduler: str = "fcfs"           # "fcfs" (Scheduler) or "priority" (PriorityScheduler)
+    num_priorities: int = 4           # priorities drawn in [0, num_priorities) for "priority"
 
 
 class Replay:
@@ -75,13 +88,19 @@ class Replay:
         rng = np.random.default_rng(c.seed)
         prompts = rng.integers(c.prompt_lo, c.prompt_hi + 1, size=c.num_requests)
         outputs = rng.integers(c.output_lo, c.output_hi + 1, size=c.num_requests)
-        self.sched = Scheduler(SchedulerConfig(
+        if c.scheduler not in ("fcfs", "priority"):
+            raise ValueError(f"unknown scheduler {c.scheduler!r}")
+        sched_cls = PriorityScheduler if c.scheduler == "priority" else Scheduler
+        self.sched = sched_cls(SchedulerConfig(
             max_num_seqs=c.max_num_seqs, max_num_batched_tokens=c.max_num_batched_tokens,
             block_size=c.block_size, num_blocks=c.num_blocks, max_model_len=c.max_model_len,
             seed=c.seed))
+        prio = (np.random.default_rng(c.seed + 7).integers(0, c.num_priorities, size=c.num_requests)
+                if c.scheduler == "priority" else np.zeros(c.num_requests, dtype=np.int64))
         self.requests = []
         for i in range(c.num_requests):
-            s = Sequence(synth.token_ids(int(prompts[i]), c.seed * 1000 + i), max_tokens=int(outputs[i]))
+            s = Sequence(synth.token_ids(int(prompts[i]), c.seed * 1000 + i), max_tokens=int(outputs[i]),
+                         priority=int(prio[i]))
             self.requests.append(s)
             self.sched.add(s)
         self.token_rng = np.random.default_rng(c.seed + 1)
@@ -125,7 +144,9 @@ class Replay:
         self.step_idx = 0
         self.stats = dict(steps=0, prefill_steps=0, decode_steps=0, prefill_tokens=0,
                           decode_tokens=0, decode_kv_bytes=0, launches=0, graph_steps=0,
-                          graph_captures=0)
+                          graph_captures=0, prefill_pairs=0, decode_context_tokens=0)
+        self.host_s = 0.0          # host time inside step()
+        self.step_events = []      # (start, end) CUDA events of each step's device work
         self.samples = {}          # (step, layer) -> captured output and the step's metadata
         self.sample_at = set()     # (step, layer) pairs to capture (needs record=True)
         self.snap = {}             # step -> slot_writer after that step's stores
@@ -218,8 +239,11 @@ class Replay:
     def step(self) -> bool:
         if self.sched.is_finished():
             return False
+        t_host = time.perf_counter()
         c, ops = self.cfg, self.ops
         seqs, is_prefill = self.sched.schedule()
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev0.record()
         bs = c.block_size
         if is_prefill:
             md = prepare_prefill(seqs, bs)
@@ -228,6 +252,9 @@ class Replay:
                                                   md.cu_seqlens_k, md.block_tables])
             self.stats["prefill_steps"] += 1
             self.stats["prefill_tokens"] += n
+            ql = np.diff(md.cu_seqlens_q).astype(np.int64)
+            kl = np.diff(md.cu_seqlens_k).astype(np.int64)
+            self.stats["prefill_pairs"] += int((ql * (kl - ql) + ql * (ql + 1) // 2).sum())
         else:
             md = prepare_decode(seqs, bs)
             n = len(seqs)
@@ -238,6 +265,7 @@ class Replay:
                 self.ws = torch.empty(need, dtype=torch.uint8, device=self.device)
             self.stats["decode_steps"] += 1
             self.stats["decode_tokens"] += n
+            self.stats["decode_context_tokens"] += int(md.context_lens.sum())
             self.stats["decode_kv_bytes"] += int(md.context_lens.sum()) * c.num_kv_heads * \
                 c.head_dim * 4 * c.num_layers
         out = self.out[:n]
@@ -274,6 +302,9 @@ class Replay:
                 n, c.num_q_heads, c.num_kv_heads, c.head_dim, md.max_context_len) > 0
         # prefill: store + attention; decode: the fused store + decode, and the merge
         self.stats["launches"] += c.num_layers * (2 if is_prefill else (2 if split else 1))
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev1.record()
+        self.step_events.append((ev0, ev1))
         if self.record:
             sm = md.slot_mapping.astype(np.int64)
             self.slot_writer[sm, 0] = self.step_idx
@@ -284,6 +315,7 @@ class Replay:
         self.sched.postprocess(seqs, toks)
         self.stats["steps"] += 1
         self.step_idx += 1
+        self.host_s += time.perf_counter() - t_host
         return True
 
     def run(self, max_steps=0):
@@ -299,7 +331,9 @@ class Replay:
         wall = time.perf_counter() - t0
         st = dict(self.stats)
         st["wall_s"] = wall
-        st["gpu_s"] = e0.elapsed_time(e1) / 1e3
+        st["gpu_s"] = e0.elapsed_time(e1) / 1e3          # span from the first to the last launch
+        st["gpu_busy_s"] = sum(a.elapsed_time(b) for a, b in self.step_events) / 1e3
+        st["host_s"] = self.host_s
         st["preemptions"] = self.sched.num_preemptions
         st["prefix_hit_tokens"] = self.sched.block_manager.prefix_hit_tokens
         st["finished"] = sum(1 for s in self.requests if s.is_finished)
@@ -316,11 +350,15 @@ def run_replay_bench(torch_mod=None, max_steps=0, cfg: ReplayConfig | None = Non
     return {
         "tokens_per_s": round(tokens / st["wall_s"], 1),
         "tokens": tokens, "wall_s": round(st["wall_s"], 3), "gpu_s": round(st["gpu_s"], 3),
+        "gpu_busy_s": round(st["gpu_busy_s"], 3), "host_s": round(st["host_s"], 3),
+        "host_over_gpu": round(st["host_s"] / st["gpu_busy_s"], 3) if st["gpu_busy_s"] else None,
+        "prefill_pairs": st["prefill_pairs"], "decode_context_tokens": st["decode_context_tokens"],
         "steps": st["steps"], "prefill_steps": st["prefill_steps"], "decode_steps": st["decode_steps"],
         "prefill_tokens": st["prefill_tokens"], "decode_tokens": st["decode_tokens"],
         "preemptions": st["preemptions"], "prefix_hit_tokens": st["prefix_hit_tokens"],
         "finished": st["finished"], "requests": cfg.num_requests, "launches": st["launches"],
         "graphs": graphs, "graph_steps": st["graph_steps"], "graph_captures": st["graph_captures"],
+        "scheduler": cfg.scheduler,
         "decode_kv_GBs": round(st["decode_kv_bytes"] / st["wall_s"] / 1e9, 1),
         "config": {"layers": cfg.num_layers, "heads": f"{cfg.num_q_heads}/{cfg.num_kv_heads}",
                    "head_dim": cfg.head_dim, "block_size": cfg.block_size,

@@ -31,15 +31,12 @@ def test_prefill_long_uncached(cuda_device):
 
 def test_prefix_cached_prefill_workload(cuda_device):
     """16 seqs, 8 fresh U[256,2048], 8 sharing a 1024-token hash-cached prefix;
-    28/4 heads, D 128, block 256.  Sampled sequences checked against the oracle."""
+    28/4 heads, D 128, block 256.  Every sequence checked against the oracle."""
     w = PrefixPrefillWorkload(seed=synth.SEED_BASE + 4).upload("cuda")
     assert sum(1 for c in w.cached if c == 1024) == 8          # the 8 prefix hits
     out = w.step().clone()
     torch.cuda.synchronize()
-    seqs = [0, 3, 8, 15]
-    ref = oracle_prefix_prefill(w, seqs)
-    rows = rows_of(w.md.cu_seqlens_q, seqs)
-    compare(out[torch.from_numpy(rows).cuda()], ref, "prefix prefill")
+    compare(out, oracle_prefix_prefill(w), "prefix prefill")
 
 
 def test_shared_prefix_equals_private_copy(cuda_device):
@@ -111,3 +108,26 @@ def test_prefill_checked_mode(cuda_device):
                        torch.from_numpy(c.block_tables).cuda(), err_flag=flag)
     torch.cuda.synchronize()
     assert int(flag.item()) & ops.FLAG_LEN_OOB
+
+
+@pytest.mark.parametrize("hq,hkv,d", [(12, 4, 128), (40, 2, 128), (8, 8, 128), (14, 2, 64)])
+def test_prefill_group_packing(cuda_device, hq, hkv, d):
+    """Query tiles pack floor(128 / G) queries x the G heads of a KV head as MMA rows:
+    groups of 3 (126 rows), 20 (120 rows), 1 (128 rows) and 7 at head_dim 64, with
+    ragged lengths, cached prefixes and a sequence with no new query."""
+    cached = [0, 5, 300, 0, 1000, 17]
+    new = [1, 50, 0, 257, 40, 700]
+    c = PrefillCase(cached, new, hq=hq, hkv=hkv, d=d, bs=64, seed=40 + hq + d)
+    out = c.run_gpu()
+    compare(out, c.oracle_prefill(), f"prefill {hq}/{hkv} d{d}")
+
+
+def test_prefill_many_sequences(cuda_device):
+    """More work units than SMs: each persistent CTA walks many units."""
+    rng = np.random.default_rng(99)
+    new = rng.integers(1, 200, size=300).tolist()
+    cached = rng.integers(0, 300, size=300).tolist()
+    c = PrefillCase(cached, new, hq=16, hkv=8, d=128, bs=16, seed=12)
+    out = c.run_gpu()
+    seqs = list(range(0, 300, 7))
+    compare(out[torch.from_numpy(c.rows_of(seqs)).cuda()], c.oracle_prefill(seqs), "many seqs")

@@ -156,3 +156,32 @@ def test_full_trace_graphs_sampled(cuda_device):
         check_sample(rp, *key, max_seqs=6)
         checked += 1
     assert checked >= 4
+
+
+def test_small_trace_priority_scheduler(cuda_device):
+    """The small trace through PriorityScheduler (seeded priorities 0..3): every step and
+    layer against the oracle; admission order follows priority, then arrival."""
+    from dataclasses import replace
+    cfg = replace(_small_cfg(), scheduler="priority", num_priorities=4)
+    rp = Replay(cfg, record="all")
+    first_prefill = None
+    orig = rp.sched.schedule
+
+    def schedule():
+        nonlocal first_prefill
+        seqs, is_prefill = orig()
+        if is_prefill and first_prefill is None:
+            first_prefill = [s.priority for s in seqs]
+        return seqs, is_prefill
+
+    rp.sched.schedule = schedule
+    st = rp.run()
+    assert st["finished"] == cfg.num_requests
+    assert len({s.priority for s in rp.requests}) > 1
+    # the first batch admits the highest priorities first
+    assert first_prefill == sorted(first_prefill, reverse=True)
+    assert max(first_prefill) == max(s.priority for s in rp.requests)
+    for (step, layer) in sorted(rp.samples):
+        check_sample(rp, step, layer)
+    assert rp.sched.block_manager.num_free_blocks == cfg.num_blocks
+    assert st["gpu_busy_s"] > 0 and st["host_s"] > 0

@@ -6,13 +6,14 @@ library offers a decode entry point whose split-K scratch is its own fixed
 16 MiB device array.  Checked here through the C ABI against pa_decode with a
 caller workspace, on two calls in a row (the second reuses the array with the
 first call's contents still in it), within the attention tolerance the other
-tests use.  This file is collected last so a stop at the first failure has
+tests use, with a checked-mode error flag that must stay 0.  A case short
+enough to need no scratch at all (one partition) goes through the same entry
+point.  This file is collected last so a stop at the first failure has
 already run everything else; it also passes alone in a fresh process.
 """
 
 from __future__ import annotations
 
-import numpy as np
 import pytest
 import torch
 
@@ -29,34 +30,41 @@ def _close(a: torch.Tensor, b: torch.Tensor):
     assert float(err.max()) <= TOL_MAX and float(err.mean()) <= TOL_MEAN
 
 
-def test_noalloc_decode_matches_pa_decode(cuda_device):
+def _twice_against_pa_decode(w, expect_scratch: bool):
     from paged_kv_attention_35_b200 import ops
-    w = DecodeWorkload.from_spec(synth.WORKLOADS["qwen3_0p6b_decode"]).upload("cuda")
     need = ops.decode_workspace_size(w.B, w.hq, w.hkv, w.d, w.max_context_len)
-    assert 0 < need <= ops.NOALLOC_SCRATCH_BYTES          # the split-K path is exercised
+    assert (0 < need <= ops.NOALLOC_SCRATCH_BYTES) if expect_scratch else need == 0
     ref = w.step().clone()                                 # pa_decode, caller workspace
     torch.cuda.synchronize()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
     outs = []
     for _ in range(2):
         out = torch.full_like(ref, float("nan"))
-        ops.decode_noalloc(w.d_q, w.kc, w.vc, w.d_bt, w.d_cl, w.max_context_len, out=out)
+        ops.decode_noalloc(w.d_q, w.kc, w.vc, w.d_bt, w.d_cl, w.max_context_len, out=out,
+                           err_flag=err)
         torch.cuda.synchronize()
+        assert int(err.item()) == 0
         _close(out, ref)
         outs.append(out)
     _close(outs[1], outs[0])
 
 
+def test_noalloc_decode_matches_pa_decode(cuda_device):
+    w = DecodeWorkload.from_spec(synth.WORKLOADS["qwen3_0p6b_decode"]).upload("cuda")
+    _twice_against_pa_decode(w, expect_scratch=True)       # the split-K path
+
+
 def test_noalloc_decode_other_shape_after_first(cuda_device):
     """A second workload (7B-GQA shape, block 16) through the same shared scratch."""
-    from paged_kv_attention_35_b200 import ops
     lens = synth.uniform_lengths(64, 512, 4096, 77).tolist()
     w = DecodeWorkload(lens, 28, 4, 128, 16, seed=77).upload("cuda")
-    ref = w.step().clone()
-    for _ in range(2):
-        out = torch.empty_like(ref)
-        ops.decode_noalloc(w.d_q, w.kc, w.vc, w.d_bt, w.d_cl, w.max_context_len, out=out)
-        torch.cuda.synchronize()
-        _close(out, ref)
+    _twice_against_pa_decode(w, expect_scratch=True)
+
+
+def test_noalloc_decode_without_scratch(cuda_device):
+    """The tiny decode step (4 seqs, contexts <= 255) fits one partition: no scratch used."""
+    w = DecodeWorkload.from_spec(synth.WORKLOADS["tiny_decode"]).upload("cuda")
+    _twice_against_pa_decode(w, expect_scratch=False)
 
 
 def test_noalloc_rejects_sizes_beyond_the_scratch(cuda_device):
