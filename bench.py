@@ -472,7 +472,7 @@ def secondary(torch, args, timer, pk):
         out["trace_replay"] = run_replay_bench(torch, max_steps=args.replay_steps, graphs=False)
         g = run_replay_bench(torch, max_steps=args.replay_steps, graphs=True)
         out["trace_replay_graphs"] = {k: g[k] for k in (
-            "tokens_per_s", "wall_s", "gpu_busy_s", "host_s", "steps", "graph_steps",
+            "tokens_per_s", "wall_s", "gpu_busy_s", "host_s", "host_wait_s", "steps", "graph_steps",
             "graph_captures", "decode_kv_GBs")}
         torch.cuda.empty_cache()
     return out
@@ -490,12 +490,14 @@ def only(args):
         tf = w.flops() / (attn_ms * 1e-3) / 1e12
         res = {"workload": "prefix_prefill", "attn_ms": round(attn_ms, 4), "TFLOPs": round(tf, 1),
                "frac_bf16_peak": round(tf / pk["bf16_tflops"], 4)}
-    elif args.only == "decode_gqa":
-        w = DecodeWorkload.from_spec(synth.WORKLOADS["gqa7b_decode"]).upload("cuda")
+    elif args.only == "decode":
+        w = DecodeWorkload.from_spec(synth.WORKLOADS[args.workload],
+                                     block_size=args.block_size or None).upload("cuda")
         r = bench_decode(torch, w, args.steps, args.warmup, timer, partition=args.partition)
         gbs = w.kv_bytes() / (r["decode_ms"] * 1e-3) / 1e9
-        res = {"workload": "gqa7b_decode", "decode_ms": round(r["decode_ms"], 4),
-               "decode_GBs": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4)}
+        res = {"workload": args.workload, "block_size": w.bs, "step_ms": round(r["step_ms"], 4),
+               "decode_ms": round(r["decode_ms"], 4), "decode_GBs": round(gbs, 1),
+               "frac_hbm": round(gbs / pk["hbm_gbs"], 4)}
     elif args.only == "store":
         nbytes, ms = bench_store_large(torch, args.steps, args.warmup, timer)
         res = {"workload": "store_kvcache_65536", "ms": round(ms, 4),
@@ -762,7 +764,8 @@ def main():
     ap.add_argument("--replay-steps", type=int, default=0)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--graphs", action="store_true", help="--only replay: graph-replayed decode steps")
-    ap.add_argument("--only", choices=["prefill", "decode_gqa", "store", "replay"], default=None,
+    ap.add_argument("--block-size", type=int, default=0, help="--only decode: pool block size")
+    ap.add_argument("--only", choices=["prefill", "decode", "store", "replay"], default=None,
                     help="time one secondary workload alone (for profiling) and print its JSON")
     args = ap.parse_args()
     if args.warmup < 3:

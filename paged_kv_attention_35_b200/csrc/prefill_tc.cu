@@ -17,18 +17,22 @@
 // of 128.
 //
 // Work unit = two consecutive query tiles (A = the later, B) of one
-// (sequence, KV head), reading the same K/V tiles.  Units are enumerated as
-// (pair from the end of the sequence, sequence, KV head), KV head fastest, so
-// the longest pairs come first and units that share K/V run side by side.
-// The kernel is persistent: one CTA per SM walks units blockIdx.x,
-// blockIdx.x + gridDim.x, ...; the K/V ring streams across unit boundaries and
-// the next unit's Q and first S overlap the current unit's epilogue.
+// (sequence, KV head), reading the same K/V tiles; its cost is the number of
+// KV tiles tile A reads.  The kernel is persistent (one CTA per SM).  Units
+// are listed from the most KV tiles to the fewest (bucket = tile A's KV tiles;
+// within a bucket by sequence, pair, KV head) and dealt out in a snake: CTA c
+// of G takes list positions c, 2G-1-c, 2G+c, 4G-1-c, ..., so the expensive
+// units go first and every CTA ends close to the mean.  Each role's warp walks
+// this list on its own (32 sequences per step, warp prefix sums; the bucket
+// of a pair follows in closed form from the sequence's lengths).  The K/V
+// ring streams across unit boundaries and the next unit's Q and first S
+// overlap the current unit's epilogue.
 //
 // Roles (10 warps):
-//   warp 8   producer: Q tiles (one box per head-dim half) into two Q buffers,
-//            then 128-key K and V tiles (one box per physical-block chunk,
-//            128-byte swizzle) into a 5-slot ring; zeroes the V rows past a
-//            unit's last key (stale pool rows may hold NaN).
+//   warp 8   producer: stages the unit's block-table entries in shared memory
+//            (one round trip), then Q tiles (one box per head-dim half) into
+//            two Q buffers and 128-key K and V tiles (one box per
+//            physical-block chunk, 128-byte swizzle) into a 5-slot ring.
 //   warp 9   MMA issuer (one thread): S_t(j) = Q_t K_j^T into tile t's TMEM S
 //            buffer (M=128, N=128, K=16 steps); O_t += P_t(j) V_j with P read
 //            from TMEM (TS form, B = V MN-major); tiles A and B interleaved so
@@ -40,6 +44,9 @@
 //            of the exponentials is evaluated on the FMA pipe (exp2_poly2) so
 //            the MUFU unit is not the only one doing them; P as bf16 pairs
 //            written back over the S columns; epilogue O / l -> bf16 -> global.
+//            Tile A's warps also zero the last V tile's rows past the unit's
+//            last key before handing over that tile's P (stale pool rows may
+//            hold NaN, and 0 * NaN = NaN in P V).
 // TMEM: 512 columns (S_A/P_A | O_A | S_B/P_B | O_B).  MMAs of one thread run
 // in issue order, so the next S never overwrites P before P V has read it, and
 // a unit's first P V into O_t is issued only after tile t's softmax warps,
@@ -76,51 +83,125 @@ struct PrefillTcParams {
   int block_size, log2_bs, box_rows;
   int num_blocks, num_slots;
   int max_seqlen_q, max_seqlen_k, total_q;
-  int64_t total_units;             // pairs x sequences x KV heads (some empty)
+  int buckets;                     // KV tiles of the longest tile: ceil(max_seqlen_k / 128)
   float scale_log2;
   int32_t* err_flag;
 };
 
 // One work unit: tiles A (t = 0) and B (t = 1) of a (sequence, KV head).
 struct TcUnit {
-  int kvh, q_start, q_len, k_len, cached;
+  int seq, kvh, q_start, q_len, k_len, cached;
   int q0[2];        // first query of tile t within the sequence
   int nt[2];        // KV tiles tile t reads (nt[1] == 0: no tile B)
   int kv_end;       // keys tile A reads (tile B reads no more)
 };
 
-// 1: a unit with work, 0: an empty slot, -1: invalid sequence lengths.
-__device__ __forceinline__ int decode_unit(const PrefillTcParams& p, int64_t idx, TcUnit& u) {
-  const int kvh = (int)(idx % p.hkv);
-  const int64_t r = idx / p.hkv;
-  const int seq = (int)(r % p.num_seqs);
-  const int pp = (int)(r / p.num_seqs);
-  const int cq0 = __ldg(p.cu_q + seq), cq1 = __ldg(p.cu_q + seq + 1);
-  const int ck0 = __ldg(p.cu_k + seq), ck1 = __ldg(p.cu_k + seq + 1);
-  const int q_len = cq1 - cq0, k_len = ck1 - ck0;
-  if (!(cq0 >= 0 && q_len >= 0 && cq1 <= p.total_q && k_len >= q_len &&
-        q_len <= p.max_seqlen_q && k_len <= p.max_seqlen_k && k_len <= p.max_blocks * p.block_size))
-    return pp == 0 && kvh == 0 ? -1 : 0;
-  const int T = (q_len + p.qpt - 1) / p.qpt;
-  if (2 * pp >= T) return 0;
-  u.kvh = kvh;
-  u.q_start = cq0;
-  u.q_len = q_len;
-  u.k_len = k_len;
-  u.cached = k_len - q_len;
-  const int ta = T - 1 - 2 * pp, tb = ta - 1;
-  u.q0[0] = ta * p.qpt;
-  u.kv_end = min(k_len, u.cached + min(q_len, u.q0[0] + p.qpt));
-  u.nt[0] = (u.kv_end + kTcKeys - 1) / kTcKeys;
-  if (tb >= 0) {
-    u.q0[1] = tb * p.qpt;
-    const int e = min(k_len, u.cached + min(q_len, u.q0[1] + p.qpt));
-    u.nt[1] = (e + kTcKeys - 1) / kTcKeys;
-  } else {
-    u.q0[1] = 0;
-    u.nt[1] = 0;
+struct TcSeq {
+  int q_start, q_len, k_len, T, P;   // T query tiles, P pairs
+  bool ok;
+};
+
+__device__ __forceinline__ TcSeq tc_seq(const PrefillTcParams& p, int s) {
+  TcSeq r;
+  const int cq0 = __ldg(p.cu_q + s), cq1 = __ldg(p.cu_q + s + 1);
+  const int ck0 = __ldg(p.cu_k + s), ck1 = __ldg(p.cu_k + s + 1);
+  r.q_start = cq0;
+  r.q_len = cq1 - cq0;
+  r.k_len = ck1 - ck0;
+  r.ok = cq0 >= 0 && r.q_len >= 0 && cq1 <= p.total_q && r.k_len >= r.q_len &&
+         r.q_len <= p.max_seqlen_q && r.k_len <= p.max_seqlen_k &&
+         r.k_len <= p.max_blocks * p.block_size;
+  r.T = r.ok ? (r.q_len + p.qpt - 1) / p.qpt : 0;
+  r.P = (r.T + 1) / 2;
+  return r;
+}
+
+// First pair (0 = the sequence's last two tiles) whose tile A reads at most b
+// KV tiles, or P when none does.  Pair pp's tile A ends at query
+// min(q_len, (T - 2 pp) qpt), so it reads ceil((cached + that) / 128) KV
+// tiles, which falls as pp grows.
+__device__ __forceinline__ int tc_first_pair(const TcSeq& q, int b, int qpt) {
+  const int cached = q.k_len - q.q_len;
+  if (cached + q.q_len <= b * kTcKeys) return 0;
+  const int R = b * kTcKeys - cached;
+  if (R < 0) return q.P;
+  return min(max((q.T - R / qpt + 1) / 2, 1), q.P);
+}
+
+// The unit list, walked by one warp (every lane calls find with the same,
+// increasing positions; the results are warp-uniform).
+struct TcWalk {
+  int b;         // current bucket
+  int s0;        // first sequence of the current window of 32
+  int64_t base;  // list position of the window's first unit
+  __device__ __forceinline__ void init(const PrefillTcParams& p) {
+    b = p.buckets;
+    s0 = 0;
+    base = 0;
   }
-  return 1;
+  // Fills u with the unit at list position pos; false past the end.  With
+  // `report`, invalid sequence lengths raise PA_FLAG_LEN_OOB (once per CTA).
+  __device__ __forceinline__ bool find(const PrefillTcParams& p, int64_t pos, int lane, bool report,
+                                       TcUnit& u) {
+    while (b > 0) {
+      const int s = s0 + lane;
+      int cnt = 0, lo = 0;
+      TcSeq q{};
+      if (s < p.num_seqs) {
+        q = tc_seq(p, s);
+        if (!q.ok && report && b == p.buckets) raise_flag(p.err_flag, PA_FLAG_LEN_OOB);
+        if (q.P > 0) {
+          lo = tc_first_pair(q, b, p.qpt);
+          cnt = (tc_first_pair(q, b - 1, p.qpt) - lo) * p.hkv;
+        }
+      }
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      if (pos < base + total) {
+        const int l = __ffs(__ballot_sync(0xffffffffu, base + incl > pos)) - 1;
+        const int64_t first = base + __shfl_sync(0xffffffffu, incl - cnt, l);
+        const int off = (int)(pos - first);
+        const int pp = __shfl_sync(0xffffffffu, lo, l) + off / p.hkv;
+        u.seq = s0 + l;
+        u.kvh = off % p.hkv;
+        u.q_start = __shfl_sync(0xffffffffu, q.q_start, l);
+        u.q_len = __shfl_sync(0xffffffffu, q.q_len, l);
+        u.k_len = __shfl_sync(0xffffffffu, q.k_len, l);
+        const int T = __shfl_sync(0xffffffffu, q.T, l);
+        u.cached = u.k_len - u.q_len;
+        const int ta = T - 1 - 2 * pp, tb = ta - 1;
+        u.q0[0] = ta * p.qpt;
+        u.kv_end = u.cached + min(u.q_len, u.q0[0] + p.qpt);
+        u.nt[0] = (u.kv_end + kTcKeys - 1) / kTcKeys;
+        if (tb >= 0) {
+          u.q0[1] = tb * p.qpt;
+          u.nt[1] = (u.cached + min(u.q_len, u.q0[1] + p.qpt) + kTcKeys - 1) / kTcKeys;
+        } else {
+          u.q0[1] = 0;
+          u.nt[1] = 0;
+        }
+        return true;
+      }
+      base += total;
+      s0 += 32;
+      if (s0 >= p.num_seqs) {
+        s0 = 0;
+        --b;
+      }
+    }
+    return false;
+  }
+};
+
+// List position of this CTA's k-th unit (snake order).
+__device__ __forceinline__ int64_t tc_position(int k) {
+  const int64_t g = gridDim.x;
+  return (int64_t)(k >> 1) * 2 * g + ((k & 1) ? 2 * g - 1 - blockIdx.x : blockIdx.x);
 }
 
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
@@ -199,18 +280,20 @@ struct Exp2Poly {
   }
 };
 
+constexpr int kBtCache = 256;    // block-table entries staged per unit
+
 struct TcBars {
   uint64_t q_full[2];      // Q tile t landed
   uint64_t q_empty[2];     // the last Q_t K^T of a unit is complete: Q buffer t free
   uint64_t kv_full[kRing];
   uint64_t kv_empty[kRing];
-  uint64_t vz[kRing];      // a unit's last V tile landed in this slot and its tail is zeroed
   uint64_t s_full[2];      // per query tile (A, B)
   uint64_t p_full[2];
   uint64_t pv_done[2];
   uint64_t drain;
   uint32_t tmem;
   int abort_flag;
+  int bt[kBtCache];        // the producer's unit: its first block-table entries
 };
 
 template <int D>
@@ -240,7 +323,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int s = 0; s < kRing; ++s) {
       mbar_init(&bar->kv_full[s], 1);
       mbar_init(&bar->kv_empty[s], 1);
-      mbar_init(&bar->vz[s], 1);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bar->s_full[t], 1);
@@ -278,15 +360,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
-    uint32_t kv_i = 0, qn[2] = {0, 0}, vz_bits = 0;
+    uint32_t kv_i = 0, qn[2] = {0, 0};
     const int box = p.box_rows;
-    for (int64_t ui = blockIdx.x; ui < p.total_units; ui += gridDim.x) {
+    TcWalk walk;
+    walk.init(p);
+    for (int k = 0;; ++k) {
       TcUnit u;
-      const int st = decode_unit(p, ui, u);
-      if (st < 0 && lane == 0) raise_flag(p.err_flag, PA_FLAG_LEN_OOB);
-      if (st <= 0) continue;
+      if (!walk.find(p, tc_position(k), lane, true, u)) break;
       const int n = u.nt[0];
-      const int32_t* bt = p.block_tables + (int64_t)(ui / p.hkv % p.num_seqs) * p.max_blocks;
+      // the unit's block-table entries, staged in one round trip
+      const int32_t* bt = p.block_tables + (int64_t)u.seq * p.max_blocks;
+      const int nblk = min((u.kv_end + p.block_size - 1) >> p.log2_bs, kBtCache);
+      for (int i = lane; i < nblk; i += 32) bar->bt[i] = __ldg(bt + i);
+      __syncwarp();
       bool ok = true;
       if (lane == 0) {
         for (int t = 0; t < 2 && ok; ++t) {
@@ -309,7 +395,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           int rows[kTcKeys / 16];
           for (int b = 0; b < nbox; ++b) {
             const int t = t0 + b * box;
-            const int bid = __ldg(bt + (t >> p.log2_bs));
+            const int lb = t >> p.log2_bs;
+            const int bid = lb < kBtCache ? bar->bt[lb] : __ldg(bt + lb);
             if (bid < 0 || bid >= p.num_blocks) {
               raise_flag(p.err_flag, PA_FLAG_BLOCK_OOB);
               rows[b] = p.num_slots;                 // past the pool: TMA fills zeros
@@ -335,84 +422,63 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
       }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      if (lane != 0) kv_i += 2 * n;                 // lane 0 counted its loads above
-      if (!ok) break;
-      // zero the last V tile's rows past the unit's last key
-      const int last_valid = u.kv_end - (n - 1) * kTcKeys;
-      if (last_valid < kTcKeys) {
-        const uint32_t iv = kv_i - 1, slot = iv % kRing;
-        bool landed = true;
-        if (lane == 0) landed = tc_wait(&bar->kv_full[slot], (iv / kRing) & 1, abort_flag, p.err_flag);
-        if (!__shfl_sync(0xffffffffu, landed ? 1 : 0, 0)) break;
-        const int nrow = kTcKeys - last_valid;
-        for (int i = lane; i < nrow * 8 * kHalves; i += 32) {
-          const int hf = i / (nrow * 8);
-          const int rr = (i >> 3) % nrow;
-          *reinterpret_cast<uint4*>(sKV + slot * kTile + hf * kTcHalf + (last_valid + rr) * 128 +
-                                    (i & 7) * 16) = make_uint4(0, 0, 0, 0);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar->vz[slot]);
-        vz_bits ^= 1u << slot;
-      }
+      // lane 0 is done with this unit's staged block table before it is overwritten
+      if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idS = tc::idesc_bf16(kTcRows, kTcKeys, false, false);
-      constexpr uint32_t idO = tc::idesc_bf16(kTcRows, D, false, true);
-      // descriptors are built once; stepping K adds (byte offset / 16) to the
-      // start-address field (no carry: shared addresses stay below 256 KB)
-      const uint64_t dQ0 = tc::sdesc_sw128(smem_u32(sQ), 16, 1024);
-      const uint64_t dK0 = tc::sdesc_sw128(smem_u32(sKV), 16, 1024);
-      const uint64_t dV0 = tc::sdesc_sw128(smem_u32(sKV), kTcHalf, 1024);
-      uint32_t kv_i = 0, qc[2] = {0, 0}, pc[2] = {0, 0}, vz_bits = 0;
-      bool ok = true;
-      auto wait_kv = [&](uint32_t i) {
-        return tc_wait(&bar->kv_full[i % kRing], (i / kRing) & 1, abort_flag, p.err_flag);
-      };
-      auto issue_s = [&](int t, uint32_t kslot) {          // S_t = Q_t K^T
-        const uint64_t dQ = dQ0 + (uint64_t)((t * kTile) >> 4);
-        const uint64_t dK = dK0 + (uint64_t)((kslot * kTile) >> 4);
+    // the whole warp walks the unit list; lane 0 issues every MMA
+    constexpr uint32_t idS = tc::idesc_bf16(kTcRows, kTcKeys, false, false);
+    constexpr uint32_t idO = tc::idesc_bf16(kTcRows, D, false, true);
+    // descriptors are built once; stepping K adds (byte offset / 16) to the
+    // start-address field (no carry: shared addresses stay below 256 KB)
+    const uint64_t dQ0 = tc::sdesc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t dK0 = tc::sdesc_sw128(smem_u32(sKV), 16, 1024);
+    const uint64_t dV0 = tc::sdesc_sw128(smem_u32(sKV), kTcHalf, 1024);
+    uint32_t kv_i = 0, qc[2] = {0, 0}, pc[2] = {0, 0};
+    auto wait_kv = [&](uint32_t i) {
+      return tc_wait(&bar->kv_full[i % kRing], (i / kRing) & 1, abort_flag, p.err_flag);
+    };
+    auto issue_s = [&](int t, uint32_t kslot) {          // S_t = Q_t K^T
+      const uint64_t dQ = dQ0 + (uint64_t)((t * kTile) >> 4);
+      const uint64_t dK = dK0 + (uint64_t)((kslot * kTile) >> 4);
 #pragma unroll
-        for (int ks = 0; ks < kSteps; ++ks) {
-          const uint64_t o = (uint64_t)(((ks >> 2) * kTcHalf + (ks & 3) * 32) >> 4);
-          tc::mma_ss(tmem + 256 * t, dQ + o, dK + o, idS, ks > 0);
-        }
-        tc::commit(&bar->s_full[t]);
-      };
-      for (int64_t ui = blockIdx.x; ok && ui < p.total_units; ui += gridDim.x) {
-        TcUnit u;
-        if (decode_unit(p, ui, u) <= 0) continue;
+      for (int ks = 0; ks < kSteps; ++ks) {
+        const uint64_t o = (uint64_t)(((ks >> 2) * kTcHalf + (ks & 3) * 32) >> 4);
+        tc::mma_ss(tmem + 256 * t, dQ + o, dK + o, idS, ks > 0);
+      }
+      tc::commit(&bar->s_full[t]);
+    };
+    TcWalk walk;
+    walk.init(p);
+    for (int k = 0;; ++k) {
+      TcUnit u;
+      if (!walk.find(p, tc_position(k), lane, false, u)) break;
+      bool ok = true;
+      if (lane == 0) {
         const int n = u.nt[0];
         for (int t = 0; t < 2 && ok; ++t)
           if (u.nt[t] > 0) ok = tc_wait(&bar->q_full[t], qc[t]++ & 1, abort_flag, p.err_flag);
-        if (!ok || !wait_kv(kv_i)) break;
-        tc::fence_after_sync();
-        for (int t = 0; t < 2; ++t) {
-          if (u.nt[t] == 0) continue;
-          issue_s(t, kv_i % kRing);
-          if (u.nt[t] == 1) tc::commit(&bar->q_empty[t]);
+        if (ok) ok = wait_kv(kv_i);                       // K_0
+        if (ok) {
+          tc::fence_after_sync();
+          for (int t = 0; t < 2; ++t) {
+            if (u.nt[t] == 0) continue;
+            issue_s(t, kv_i % kRing);
+            if (u.nt[t] == 1) tc::commit(&bar->q_empty[t]);
+          }
+          tc::commit(&bar->kv_empty[kv_i % kRing]);        // K_0 consumed
         }
-        tc::commit(&bar->kv_empty[kv_i % kRing]);          // K_0 consumed
-        const bool zero_tail = u.kv_end - (n - 1) * kTcKeys < kTcKeys;
         for (int j = 0; ok && j < n; ++j) {
           const uint32_t iv = kv_i + 2 * j + 1, vslot = iv % kRing;
           const uint32_t kn = iv + 1, kslot = kn % kRing;  // K_j+1
-          // operands first (normally resident long before the softmax is done)
-          bool got;
-          if (zero_tail && j == n - 1) {
-            got = tc_wait(&bar->vz[vslot], (vz_bits >> vslot) & 1, abort_flag, p.err_flag);
-            vz_bits ^= 1u << vslot;
-          } else {
-            got = wait_kv(iv);
-          }
-          if (!got || (j + 1 < n && !wait_kv(kn))) {
+          // V_j's tail rows (last tile) are zeroed by tile A's softmax before
+          // it hands over P, so the V_j wait is the plain landing wait
+          if (!wait_kv(iv)) {
             ok = false;
             break;
           }
+          bool k_next = false;
           for (int t = 0; t < 2; ++t) {
             if (j >= u.nt[t]) continue;
             if (!tc_wait(&bar->p_full[t], pc[t]++ & 1, abort_flag, p.err_flag)) {
@@ -427,6 +493,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                          dV + (uint64_t)((ks * 2048) >> 4), idO, (j > 0 || ks > 0));
             if (j == u.nt[t] - 1) tc::commit(&bar->pv_done[t]);   // the epilogue waits on it
             if (j + 1 < u.nt[t]) {
+              if (!k_next) {                     // K_j+1 is needed only from here on
+                if (!wait_kv(kn)) {
+                  ok = false;
+                  break;
+                }
+                tc::fence_after_sync();
+                k_next = true;
+              }
               issue_s(t, kslot);
               if (j + 2 == u.nt[t]) tc::commit(&bar->q_empty[t]);
             }
@@ -437,10 +511,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         kv_i += 2 * n;
       }
+      if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+    }
+    if (lane == 0) {
       // every issued MMA finishes before TMEM is released
       tc::commit(&bar->drain);
       mbar_wait(&bar->drain, 0);
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax (warpgroup t = tile)
     const int t = warp >> 2;                       // 0: tile A, 1: tile B
@@ -451,10 +529,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const float sl2 = p.scale_log2;
     const Exp2Poly ex;
     uint32_t sc = 0, pvc = 0;
+    uint32_t kv_i = 0;                             // ring index of the unit's K_0 (tile A tracks it)
     bool ok = true;
-    for (int64_t ui = blockIdx.x; ok && ui < p.total_units; ui += gridDim.x) {
+    TcWalk walk;
+    walk.init(p);
+    for (int k = 0; ok; ++k) {
       TcUnit u;
-      if (decode_unit(p, ui, u) <= 0 || u.nt[t] == 0) continue;
+      if (!walk.find(p, tc_position(k), lane, false, u)) break;
+      const uint32_t kv_unit = kv_i;
+      kv_i += 2 * u.nt[0];
+      if (u.nt[t] == 0) continue;
       const int nt = u.nt[t], q0 = u.q0[t];
       const int limit = min(u.cached + q0 + qi, u.k_len - 1);   // last visible key of this row
       float m_ref = -INFINITY, l = 0.f;
@@ -517,6 +601,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             pk[(i >> 1) & 31] = pack_bf16(e0, e1);
           }
           tc::st32(tS + 32 * hk, pk);
+        }
+        if (t == 0 && j == nt - 1) {
+          // the unit's last V tile: zero its rows past the last key before P V reads them
+          const int last_valid = u.kv_end - j * kTcKeys;
+          if (last_valid < kTcKeys) {
+            const uint32_t iv = kv_unit + 2 * j + 1, slot = iv % kRing;
+            if (!__all_sync(0xffffffffu, tc_wait(&bar->kv_full[slot], (iv / kRing) & 1, abort_flag,
+                                                 p.err_flag))) {
+              ok = false;
+              break;
+            }
+            const int nrow = kTcKeys - last_valid;
+            for (int i = r; i < nrow * 8 * kHalves; i += kTcRows) {
+              const int hf = i / (nrow * 8);
+              const int rr = (i >> 3) % nrow;
+              *reinterpret_cast<uint4*>(sKV + slot * kTile + hf * kTcHalf + (last_valid + rr) * 128 +
+                                        (i & 7) * 16) = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+          }
         }
         {
           float a0, a1, b0, b1;
@@ -614,17 +718,20 @@ static pa_status launch_prefill_d(const PrefillArgs& a) {
   prm.max_seqlen_q = a.max_seqlen_q;
   prm.max_seqlen_k = a.max_seqlen_k;
   prm.total_q = a.total_q;
+  prm.buckets = (a.max_seqlen_k + kTcKeys - 1) / kTcKeys;
   const int64_t max_pairs = ((int64_t)(a.max_seqlen_q + qpt - 1) / qpt + 1) / 2;
-  prm.total_units = max_pairs * a.num_seqs * a.hkv;
+  const int64_t max_units = max_pairs * a.num_seqs * a.hkv;
   prm.scale_log2 = a.scale * 1.4426950408889634f;
   prm.err_flag = a.err_flag;
   // at least 120 KB so that two CTAs never share an SM (each allocates all 512
   // TMEM columns)
+  static_assert((2 + kRing) * (size_t)kTile + 1024 + sizeof(TcBars) <= 232448,
+                "prefill shared memory exceeds the 227 KB a CTA may use");
   size_t smem = (2 + kRing) * (size_t)kTile + 1024 + sizeof(TcBars);
   if (smem < 120 * 1024) smem = 120 * 1024;
   s = ensure_smem_attr((const void*)prefill_tc_kernel<D>, (int)smem, "prefill smem attribute");
   if (s != PA_OK) return s;
-  const int64_t ctas = prm.total_units < device_sm_count() ? prm.total_units : device_sm_count();
+  const int64_t ctas = max_units < device_sm_count() ? max_units : device_sm_count();
   cudaError_t e = launch_pdl(prefill_tc_kernel<D>, dim3((unsigned)ctas), dim3(kTcThreads), smem,
                              a.stream, mq, mk, mv, prm);
   if (e != cudaSuccess) {

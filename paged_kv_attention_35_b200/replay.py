@@ -25,8 +25,9 @@ On the first step of a key the layers run eagerly and the graph is captured
 for the next ones.  Prefill steps always run eagerly.
 
 Timing: ``run`` reports the wall time of the loop, the host time spent inside
-the steps (scheduling, preparation, packing, launching, postprocessing), and
-the GPU time of the steps: for each step the device time from its metadata
+the steps (scheduling, preparation, packing, launching, postprocessing) and
+how much of it was spent blocked on the GPU (a pinned staging buffer whose
+copy has not run yet), and the GPU time of the steps: for each step the device time from its metadata
 copy to its last kernel, summed (idle device time between steps, while the
 host prepares the next one, is not counted).
 
@@ -146,6 +147,7 @@ class Replay:
                           decode_tokens=0, decode_kv_bytes=0, launches=0, graph_steps=0,
                           graph_captures=0, prefill_pairs=0, decode_context_tokens=0)
         self.host_s = 0.0          # host time inside step()
+        self.host_wait_s = 0.0     # of which blocked on the GPU (a staging buffer still in use)
         self.step_events = []      # (start, end) CUDA events of each step's device work
         self.samples = {}          # (step, layer) -> captured output and the step's metadata
         self.sample_at = set()     # (step, layer) pairs to capture (needs record=True)
@@ -159,7 +161,9 @@ class Replay:
         """Pack int32 arrays into a pinned buffer and copy them to the device in one go."""
         b = self.step_idx & 1
         if self.pinned_ev[b] is not None:
+            t0 = time.perf_counter()
             self.pinned_ev[b].synchronize()        # the copy that last used this buffer is done
+            self.host_wait_s += time.perf_counter() - t0
         buf = self.pinned[b]
         views, off = [], 0
         host = buf.numpy()
@@ -201,7 +205,9 @@ class Replay:
         nb, lb = self._batch_bucket(n), self._ctx_bucket(md.max_context_len)
         b = self.step_idx & 1
         if self.g_pinned_ev[b] is not None:
+            t0 = time.perf_counter()
             self.g_pinned_ev[b].synchronize()
+            self.host_wait_s += time.perf_counter() - t0
         host = self.g_pinned[b].numpy()
         host[:nb] = -1
         host[:n] = md.slot_mapping
@@ -334,6 +340,7 @@ class Replay:
         st["gpu_s"] = e0.elapsed_time(e1) / 1e3          # span from the first to the last launch
         st["gpu_busy_s"] = sum(a.elapsed_time(b) for a, b in self.step_events) / 1e3
         st["host_s"] = self.host_s
+        st["host_wait_s"] = self.host_wait_s
         st["preemptions"] = self.sched.num_preemptions
         st["prefix_hit_tokens"] = self.sched.block_manager.prefix_hit_tokens
         st["finished"] = sum(1 for s in self.requests if s.is_finished)
@@ -351,7 +358,9 @@ def run_replay_bench(torch_mod=None, max_steps=0, cfg: ReplayConfig | None = Non
         "tokens_per_s": round(tokens / st["wall_s"], 1),
         "tokens": tokens, "wall_s": round(st["wall_s"], 3), "gpu_s": round(st["gpu_s"], 3),
         "gpu_busy_s": round(st["gpu_busy_s"], 3), "host_s": round(st["host_s"], 3),
-        "host_over_gpu": round(st["host_s"] / st["gpu_busy_s"], 3) if st["gpu_busy_s"] else None,
+        "host_wait_s": round(st["host_wait_s"], 3),
+        "host_work_over_gpu": round((st["host_s"] - st["host_wait_s"]) / st["gpu_busy_s"], 3)
+        if st["gpu_busy_s"] else None,
         "prefill_pairs": st["prefill_pairs"], "decode_context_tokens": st["decode_context_tokens"],
         "steps": st["steps"], "prefill_steps": st["prefill_steps"], "decode_steps": st["decode_steps"],
         "prefill_tokens": st["prefill_tokens"], "decode_tokens": st["decode_tokens"],
