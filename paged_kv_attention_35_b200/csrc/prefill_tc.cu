@@ -33,10 +33,11 @@
 //            (one round trip), then Q tiles (one box per head-dim half) into
 //            two Q buffers and 128-key K and V tiles (one box per
 //            physical-block chunk, 128-byte swizzle) into a 5-slot ring.
-//   warp 9   MMA issuer (one thread): S_t(j) = Q_t K_j^T into tile t's TMEM S
-//            buffer (M=128, N=128, K=16 steps); O_t += P_t(j) V_j with P read
-//            from TMEM (TS form, B = V MN-major); tiles A and B interleaved so
-//            one tile's softmax overlaps the other's MMAs.
+//   warp 9   MMA issuer (one thread): S_t(j) = Q_t K_j^T into the TMEM S
+//            columns (M=128, N=128, K=16 steps); O_t += P_t(j) V_j with P read
+//            from TMEM (TS form, B = V MN-major); per KV tile the order is
+//            S_A(j+1), P_A(j) V_j, S_B(j+1), P_B(j) V_j, so the tensor core
+//            works on one tile while the other tile's softmax runs.
 //   warps 0-3 / 4-7   softmax of tile A / B, one thread per M row (TMEM lane):
 //            causal mask on the tiles that reach past a row's last key; online
 //            softmax in the log2 domain with a lazy rescale (the reference max
@@ -47,9 +48,11 @@
 //            Tile A's warps also zero the last V tile's rows past the unit's
 //            last key before handing over that tile's P (stale pool rows may
 //            hold NaN, and 0 * NaN = NaN in P V).
-// TMEM: 512 columns (S_A/P_A | O_A | S_B/P_B | O_B).  MMAs of one thread run
-// in issue order, so the next S never overwrites P before P V has read it, and
-// a unit's first P V into O_t is issued only after tile t's softmax warps,
+// TMEM: 512 columns: S (128, shared by the tiles in turn) | P_A (64) | P_B (64) |
+// O_A | O_B.  A tile's softmax releases the S columns as soon as S is in its
+// registers, so the next Q K^T overlaps the exponentials instead of waiting
+// for P V; P_t is rewritten only after the previous P_t V has completed, and a
+// unit's first P V into O_t is issued only after tile t's softmax warps,
 // which also run its epilogue, have read the previous unit's O_t.
 // Every wait is bounded; an abort winds all roles down, drains the issued
 // MMAs and frees TMEM.
@@ -67,11 +70,13 @@ constexpr int kTcKeys = 128;     // keys per KV tile (MMA N of QK^T, K of PV)
 constexpr int kTcThreads = 320;  // 2 softmax warpgroups + producer warp + MMA warp
 constexpr int kTcHalf = kTcRows * 128;  // one 128-row x 64-element bf16 half (swizzled)
 constexpr int kRing = 5;         // K/V ring slots (K_j, V_j, K_j+1, ... in turn)
+// TMEM columns: S (shared by the two tiles in turn), P_A, P_B (bf16 pairs), O_A, O_B
+constexpr uint32_t kTmemS = 0, kTmemP = 128, kTmemO = 256;
 constexpr float kLazyRescale = 8.f;   // log2 of the largest un-rescaled growth (256x)
 
 // Exponentials evaluated by polynomial: pair k of every 8 value pairs (16
 // scores) is emulated when bit k is set.
-constexpr uint32_t kEmuPairs = 0x4A;   // pairs 1, 3, 6: 3 of 8
+constexpr uint32_t kEmuPairs = 0x0;    // none: measured faster (the MUFU is not the limiter)
 
 struct PrefillTcParams {
   __nv_bfloat16* out;
@@ -128,40 +133,50 @@ __device__ __forceinline__ int tc_first_pair(const TcSeq& q, int b, int qpt) {
   return min(max((q.T - R / qpt + 1) / 2, 1), q.P);
 }
 
-// The unit list, walked by one warp (every lane calls find with the same,
-// increasing positions; the results are warp-uniform).
+// The unit list, walked by the producer warp (every lane calls find with the
+// same, increasing positions; the results are warp-uniform).  The current
+// window's per-sequence values stay in registers until the walk moves on.
 struct TcWalk {
   int b;         // current bucket
   int s0;        // first sequence of the current window of 32
   int64_t base;  // list position of the window's first unit
+  bool have;     // the lane values below belong to (b, s0)
+  int cnt, lo, incl, total;   // this lane's sequence in the window: units, first pair, prefix
+  TcSeq q;
   __device__ __forceinline__ void init(const PrefillTcParams& p) {
     b = p.buckets;
     s0 = 0;
     base = 0;
+    have = false;
   }
   // Fills u with the unit at list position pos; false past the end.  With
   // `report`, invalid sequence lengths raise PA_FLAG_LEN_OOB (once per CTA).
   __device__ __forceinline__ bool find(const PrefillTcParams& p, int64_t pos, int lane, bool report,
                                        TcUnit& u) {
     while (b > 0) {
-      const int s = s0 + lane;
-      int cnt = 0, lo = 0;
-      TcSeq q{};
-      if (s < p.num_seqs) {
-        q = tc_seq(p, s);
-        if (!q.ok && report && b == p.buckets) raise_flag(p.err_flag, PA_FLAG_LEN_OOB);
-        if (q.P > 0) {
-          lo = tc_first_pair(q, b, p.qpt);
-          cnt = (tc_first_pair(q, b - 1, p.qpt) - lo) * p.hkv;
+      if (!have) {
+        const int s = s0 + lane;
+        cnt = 0;
+        lo = 0;
+        if (s < p.num_seqs) {
+          q = tc_seq(p, s);
+          if (!q.ok && report && b == p.buckets) raise_flag(p.err_flag, PA_FLAG_LEN_OOB);
+          if (q.P > 0) {
+            lo = tc_first_pair(q, b, p.qpt);
+            cnt = (tc_first_pair(q, b - 1, p.qpt) - lo) * p.hkv;
+          }
+        } else {
+          q = TcSeq{};
         }
-      }
-      int incl = cnt;
+        incl = cnt;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        total = __shfl_sync(0xffffffffu, incl, 31);
+        have = true;
       }
-      const int total = __shfl_sync(0xffffffffu, incl, 31);
       if (pos < base + total) {
         const int l = __ffs(__ballot_sync(0xffffffffu, base + incl > pos)) - 1;
         const int64_t first = base + __shfl_sync(0xffffffffu, incl - cnt, l);
@@ -188,6 +203,7 @@ struct TcWalk {
         return true;
       }
       base += total;
+      have = false;
       s0 += 32;
       if (s0 >= p.num_seqs) {
         s0 = 0;
@@ -221,6 +237,49 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
   }
 }
 
+// The same bounded wait as one inline-PTX loop, for waits taken while the
+// softmax holds a full S row in registers (a C++ loop there makes the
+// compiler spill the row): polls the phase, gives up when another role has
+// aborted or after kWaitLimitNs.
+__device__ __forceinline__ bool tc_wait_inline(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort_flag, int32_t* err_flag) {
+  uint32_t res;
+  asm volatile(
+      "{\n\t"
+      ".reg .pred P1;\n\t"
+      ".reg .u64 T0, T1;\n\t"
+      ".reg .u32 AB;\n\t"
+      "mov.u64 T0, %%globaltimer;\n"
+      "TCW_LOOP:\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
+      "@P1 bra TCW_DONE;\n\t"
+      "ld.volatile.shared.u32 AB, [%3];\n\t"
+      "setp.ne.u32 P1, AB, 0;\n\t"
+      "@P1 bra TCW_ABORT;\n\t"
+      "mov.u64 T1, %%globaltimer;\n\t"
+      "sub.u64 T1, T1, T0;\n\t"
+      "setp.lt.u64 P1, T1, %4;\n\t"
+      "@P1 bra TCW_LOOP;\n\t"
+      "mov.u32 %0, 0;\n\t"
+      "bra TCW_END;\n"
+      "TCW_ABORT:\n\t"
+      "mov.u32 %0, 2;\n\t"
+      "bra TCW_END;\n"
+      "TCW_DONE:\n\t"
+      "mov.u32 %0, 1;\n"
+      "TCW_END:\n\t"
+      "}"
+      : "=r"(res)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(smem_u32(const_cast<int*>(abort_flag))),
+        "l"(kWaitLimitNs)
+      : "memory");
+  if (res == 0) {
+    *abort_flag = 1;
+    raise_flag(err_flag, PA_FLAG_TIMEOUT);
+  }
+  return res == 1;
+}
+
 // Packed / 3-input fp32 arithmetic of sm_100 (halves the softmax's issue slots).
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
@@ -247,7 +306,8 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
 }
 
 // 2^x for two values on the FMA pipe.  x is clamped to >= -125 (2^-125 is
-// below anything that survives the bf16 rounding of P next to a 1), then
+// below anything that survives the bf16 rounding of P next to a 1; below the
+// clamp the result is exactly 0, as for masked scores), then
 // split as x = j + f with j the nearest integer (adding and subtracting
 // 1.5 * 2^23 rounds to an integer in the low mantissa bits) and f in
 // [-0.5, 0.5]; 2^f is a cubic whose coefficients were fitted to minimise the
@@ -277,30 +337,57 @@ struct Exp2Poly {
     f32x2_split(t, t0, t1);
     e0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
     e1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+    e0 = x0 > -125.f ? e0 : 0.f;                 // masked scores (-inf) give exactly 0
+    e1 = x1 > -125.f ? e1 : 0.f;
   }
 };
 
 constexpr int kBtCache = 256;    // block-table entries staged per unit
+constexpr int kUnitSlots = 4;    // unit descriptors the producer publishes ahead
+constexpr int kUnitReaders = 9;  // the MMA warp and the 8 softmax warps
 
 struct TcBars {
   uint64_t q_full[2];      // Q tile t landed
   uint64_t q_empty[2];     // the last Q_t K^T of a unit is complete: Q buffer t free
   uint64_t kv_full[kRing];
   uint64_t kv_empty[kRing];
-  uint64_t s_full[2];      // per query tile (A, B)
-  uint64_t p_full[2];
-  uint64_t pv_done[2];
+  uint64_t s_full[2];      // S_t is in the S columns
+  uint64_t s_free;         // the S columns have been read into registers
+  uint64_t p_full[2];      // P_t is in its TMEM columns (O_t rescaled if needed)
+  uint64_t pv_done[2];     // the last P_t V issued is complete
   uint64_t drain;
+  uint64_t unit_full[kUnitSlots];   // descriptor published (nt[0] == 0: no more units)
+  uint64_t unit_empty[kUnitSlots];  // every reader has copied it
+  TcUnit units[kUnitSlots];
   uint32_t tmem;
   int abort_flag;
   int bt[kBtCache];        // the producer's unit: its first block-table entries
 };
+
+// The k-th unit descriptor the producer published, read by a whole warp
+// (warp-uniform result; false when the list is over or a wait gave up).
+__device__ __forceinline__ bool tc_take_unit(TcBars* bar, uint32_t k, int lane,
+                                             volatile int* abort_flag, int32_t* err_flag,
+                                             TcUnit& u, bool& ok) {
+  const uint32_t slot = k % kUnitSlots;
+  bool got = true;
+  if (lane == 0) got = tc_wait(&bar->unit_full[slot], (k / kUnitSlots) & 1, abort_flag, err_flag);
+  if (!__shfl_sync(0xffffffffu, got ? 1 : 0, 0)) {
+    ok = false;
+    return false;
+  }
+  u = bar->units[slot];
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&bar->unit_empty[slot]);
+  return u.nt[0] > 0;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const PrefillTcParams p) {
   constexpr int kHalves = D / 64;
+  constexpr uint32_t kOCols = D;               // TMEM columns of one O accumulator
   constexpr int kTile = kHalves * kTcHalf;     // one Q, K or V tile
   constexpr int kSteps = D / 16;               // K steps of Q K^T
   extern __shared__ uint8_t smem_raw[];
@@ -330,6 +417,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&bar->pv_done[t], 1);
     }
     mbar_init(&bar->drain, 1);
+    mbar_init(&bar->s_free, 4);
+    for (int s = 0; s < kUnitSlots; ++s) {
+      mbar_init(&bar->unit_full[s], 1);
+      mbar_init(&bar->unit_empty[s], kUnitReaders);
+    }
     bar->abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmQ);
@@ -354,8 +446,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  // tile t: S at TMEM columns [256t, 256t+128) with P (bf16 pairs) over its
-  // first 64 columns once S has been read; O at [256t+128, 256t+128+D)
   const uint32_t tmem = bar->tmem;
 
   if (warp == 8) {
@@ -366,7 +456,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     walk.init(p);
     for (int k = 0;; ++k) {
       TcUnit u;
-      if (!walk.find(p, tc_position(k), lane, true, u)) break;
+      const bool more = walk.find(p, tc_position(k), lane, true, u);
+      if (!more) u.nt[0] = 0;                   // the end of this CTA's list
+      // publish the unit to the MMA and softmax warps
+      const uint32_t us = (uint32_t)k % kUnitSlots;
+      bool free_slot = true;
+      if (lane == 0 && k >= kUnitSlots)
+        free_slot = tc_wait(&bar->unit_empty[us], ((k / kUnitSlots) - 1) & 1, abort_flag, p.err_flag);
+      if (!__shfl_sync(0xffffffffu, free_slot ? 1 : 0, 0)) break;
+      if (lane == 0) {
+        bar->units[us] = u;
+        mbar_arrive(&bar->unit_full[us]);
+      }
+      if (!more) break;
       const int n = u.nt[0];
       // the unit's block-table entries, staged in one round trip
       const int32_t* bt = p.block_tables + (int64_t)u.seq * p.max_blocks;
@@ -427,7 +529,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    // the whole warp walks the unit list; lane 0 issues every MMA
+    // The warp takes the unit descriptors; lane 0 issues every MMA.  Order
+    // per KV tile j:  S_A(j+1), P_A(j) V_j, S_B(j+1), P_B(j) V_j, where each
+    // S waits only until the previous S in the shared S columns has been
+    // read into registers, and each P V until that tile's P is in TMEM.
     constexpr uint32_t idS = tc::idesc_bf16(kTcRows, kTcKeys, false, false);
     constexpr uint32_t idO = tc::idesc_bf16(kTcRows, D, false, true);
     // descriptors are built once; stepping K adds (byte offset / 16) to the
@@ -435,77 +540,79 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint64_t dQ0 = tc::sdesc_sw128(smem_u32(sQ), 16, 1024);
     const uint64_t dK0 = tc::sdesc_sw128(smem_u32(sKV), 16, 1024);
     const uint64_t dV0 = tc::sdesc_sw128(smem_u32(sKV), kTcHalf, 1024);
-    uint32_t kv_i = 0, qc[2] = {0, 0}, pc[2] = {0, 0};
+    uint32_t kv_i = 0, qc[2] = {0, 0}, pc[2] = {0, 0}, s_issued = 0;
     auto wait_kv = [&](uint32_t i) {
       return tc_wait(&bar->kv_full[i % kRing], (i / kRing) & 1, abort_flag, p.err_flag);
     };
-    auto issue_s = [&](int t, uint32_t kslot) {          // S_t = Q_t K^T
+    // S_t = Q_t K^T into the shared S columns, once the previous S there has been read
+    auto issue_s = [&](int t, uint32_t kslot) {
+      if (s_issued > 0 && !tc_wait(&bar->s_free, (s_issued - 1) & 1, abort_flag, p.err_flag))
+        return false;
+      tc::fence_after_sync();
       const uint64_t dQ = dQ0 + (uint64_t)((t * kTile) >> 4);
       const uint64_t dK = dK0 + (uint64_t)((kslot * kTile) >> 4);
 #pragma unroll
       for (int ks = 0; ks < kSteps; ++ks) {
         const uint64_t o = (uint64_t)(((ks >> 2) * kTcHalf + (ks & 3) * 32) >> 4);
-        tc::mma_ss(tmem + 256 * t, dQ + o, dK + o, idS, ks > 0);
+        tc::mma_ss(tmem + kTmemS, dQ + o, dK + o, idS, ks > 0);
       }
       tc::commit(&bar->s_full[t]);
+      ++s_issued;
+      return true;
     };
-    TcWalk walk;
-    walk.init(p);
-    for (int k = 0;; ++k) {
+    // O_t += P_t V_j (the last tile: only the 16-key steps before kv_end)
+    auto issue_pv = [&](const TcUnit& u, int t, int j, uint32_t vslot) {
+      if (!tc_wait(&bar->p_full[t], pc[t]++ & 1, abort_flag, p.err_flag)) return false;
+      tc::fence_after_sync();
+      const uint64_t dV = dV0 + (uint64_t)((vslot * kTile) >> 4);
+      const int nks = j == u.nt[0] - 1 ? (u.kv_end - j * kTcKeys + 15) / 16 : kTcKeys / 16;
+#pragma unroll
+      for (int ks = 0; ks < kTcKeys / 16; ++ks)
+        if (ks < nks)
+          tc::mma_ts(tmem + kTmemO + kOCols * t, tmem + kTmemP + 64 * t + ks * 8,
+                     dV + (uint64_t)((ks * 2048) >> 4), idO, (j > 0 || ks > 0));
+      tc::commit(&bar->pv_done[t]);
+      return true;
+    };
+    for (uint32_t k = 0;; ++k) {
       TcUnit u;
-      if (!walk.find(p, tc_position(k), lane, false, u)) break;
       bool ok = true;
+      if (!tc_take_unit(bar, k, lane, abort_flag, p.err_flag, u, ok)) break;
       if (lane == 0) {
-        const int n = u.nt[0];
+        const int n = u.nt[0], nb = u.nt[1];
         for (int t = 0; t < 2 && ok; ++t)
           if (u.nt[t] > 0) ok = tc_wait(&bar->q_full[t], qc[t]++ & 1, abort_flag, p.err_flag);
         if (ok) ok = wait_kv(kv_i);                       // K_0
         if (ok) {
           tc::fence_after_sync();
-          for (int t = 0; t < 2; ++t) {
-            if (u.nt[t] == 0) continue;
-            issue_s(t, kv_i % kRing);
-            if (u.nt[t] == 1) tc::commit(&bar->q_empty[t]);
-          }
-          tc::commit(&bar->kv_empty[kv_i % kRing]);        // K_0 consumed
+          ok = issue_s(0, kv_i % kRing);
+          if (ok && n == 1) tc::commit(&bar->q_empty[0]);
         }
+        if (ok && nb > 0) {
+          ok = issue_s(1, kv_i % kRing);
+          if (ok && nb == 1) tc::commit(&bar->q_empty[1]);
+        }
+        if (ok) tc::commit(&bar->kv_empty[kv_i % kRing]);  // K_0 consumed
         for (int j = 0; ok && j < n; ++j) {
           const uint32_t iv = kv_i + 2 * j + 1, vslot = iv % kRing;
           const uint32_t kn = iv + 1, kslot = kn % kRing;  // K_j+1
-          // V_j's tail rows (last tile) are zeroed by tile A's softmax before
-          // it hands over P, so the V_j wait is the plain landing wait
-          if (!wait_kv(iv)) {
-            ok = false;
-            break;
+          if (j + 1 < n) {
+            if (!wait_kv(kn)) { ok = false; break; }
+            if (!issue_s(0, kslot)) { ok = false; break; }
+            if (j + 2 == n) tc::commit(&bar->q_empty[0]);
           }
-          bool k_next = false;
-          for (int t = 0; t < 2; ++t) {
-            if (j >= u.nt[t]) continue;
-            if (!tc_wait(&bar->p_full[t], pc[t]++ & 1, abort_flag, p.err_flag)) {
-              ok = false;
-              break;
+          // V_j's tail rows (last tile) are zeroed by tile A's softmax before it
+          // hands over P, so the V_j wait is the plain landing wait
+          if (!wait_kv(iv)) { ok = false; break; }
+          tc::fence_after_sync();
+          if (!issue_pv(u, 0, j, vslot)) { ok = false; break; }
+          if (j < nb) {
+            if (j + 1 < nb) {
+              if (!issue_s(1, kslot)) { ok = false; break; }
+              if (j + 2 == nb) tc::commit(&bar->q_empty[1]);
             }
-            tc::fence_after_sync();
-            const uint64_t dV = dV0 + (uint64_t)((vslot * kTile) >> 4);
-#pragma unroll
-            for (int ks = 0; ks < kTcKeys / 16; ++ks)
-              tc::mma_ts(tmem + 256 * t + 128, tmem + 256 * t + ks * 8,
-                         dV + (uint64_t)((ks * 2048) >> 4), idO, (j > 0 || ks > 0));
-            if (j == u.nt[t] - 1) tc::commit(&bar->pv_done[t]);   // the epilogue waits on it
-            if (j + 1 < u.nt[t]) {
-              if (!k_next) {                     // K_j+1 is needed only from here on
-                if (!wait_kv(kn)) {
-                  ok = false;
-                  break;
-                }
-                tc::fence_after_sync();
-                k_next = true;
-              }
-              issue_s(t, kslot);
-              if (j + 2 == u.nt[t]) tc::commit(&bar->q_empty[t]);
-            }
+            if (!issue_pv(u, 1, j, vslot)) { ok = false; break; }
           }
-          if (!ok) break;
           tc::commit(&bar->kv_empty[vslot]);                 // V_j consumed
           if (j + 1 < n) tc::commit(&bar->kv_empty[kslot]);  // K_j+1 consumed
         }
@@ -525,17 +632,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int r = threadIdx.x & 127;               // M row = TMEM lane
     const int qi = r / p.group, hh = r - qi * p.group;   // query within the tile, head in the group
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + 256 * t + lane_off, tO = tS + 128;
+    const uint32_t tS = tmem + kTmemS + lane_off;
+    const uint32_t tP = tmem + kTmemP + 64 * t + lane_off;
+    const uint32_t tO = tmem + kTmemO + kOCols * t + lane_off;
     const float sl2 = p.scale_log2;
     const Exp2Poly ex;
     uint32_t sc = 0, pvc = 0;
     uint32_t kv_i = 0;                             // ring index of the unit's K_0 (tile A tracks it)
     bool ok = true;
-    TcWalk walk;
-    walk.init(p);
-    for (int k = 0; ok; ++k) {
+    for (uint32_t k = 0; ok; ++k) {
       TcUnit u;
-      if (!walk.find(p, tc_position(k), lane, false, u)) break;
+      if (!tc_take_unit(bar, k, lane, abort_flag, p.err_flag, u, ok)) break;
       const uint32_t kv_unit = kv_i;
       kv_i += 2 * u.nt[0];
       if (u.nt[t] == 0) continue;
@@ -543,8 +650,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int limit = min(u.cached + q0 + qi, u.k_len - 1);   // last visible key of this row
       float m_ref = -INFINITY, l = 0.f;
       for (int j = 0; j < nt; ++j) {
-        // S_t(j) complete implies every earlier MMA of this CTA -- P V of tile j-1
-        // included -- is complete: O may be rescaled and the S/P columns reused.
         if (!__all_sync(0xffffffffu, tc_wait(&bar->s_full[t], sc++ & 1, abort_flag, p.err_flag))) {
           ok = false;
           break;
@@ -554,6 +659,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tc::ld32(tS + c * 32, reinterpret_cast<uint32_t*>(sv) + c * 32);
         tc::wait_ld();
+        // S is in registers: the next Q K^T may overwrite the S columns
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->s_free);
         const int t0 = j * kTcKeys;
         if (t0 + kTcKeys - 1 > limit) {            // tile reaches past the row's last key: mask
           const int lim = limit - t0;
@@ -582,11 +691,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
         const uint64_t sc2 = f32x2(sl2, sl2), nm2 = f32x2(neg_m, neg_m);
         uint64_t rs2[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
-        // P in two halves of 64 keys, each stored as 32 bf16 pairs over the S
-        // columns it came from (S is already in registers)
+        // P as 64 bf16 pairs (kept in registers until the previous P_t V is done)
+        uint32_t pk[kTcKeys / 2];
 #pragma unroll
         for (int hk = 0; hk < 2; ++hk) {
-          uint32_t pk[32];
 #pragma unroll
           for (int i = 64 * hk; i < 64 * hk + 64; i += 2) {
             float x0, x1, e0, e1;
@@ -598,21 +706,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               e1 = fast_exp2(x1);
             }
             rs2[(i >> 1) & 1] = fadd2(rs2[(i >> 1) & 1], f32x2(e0, e1));
-            pk[(i >> 1) & 31] = pack_bf16(e0, e1);
+            pk[i >> 1] = pack_bf16(e0, e1);
           }
-          tc::st32(tS + 32 * hk, pk);
         }
+        // the previous P_t V must be complete before P_t is overwritten and O_t rescaled
+        if (j > 0 && !__all_sync(0xffffffffu,
+                                 tc_wait_inline(&bar->pv_done[t], pvc++ & 1, abort_flag, p.err_flag))) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        tc::st32(tP, pk);
+        tc::st32(tP + 32, pk + 32);
         if (t == 0 && j == nt - 1) {
-          // the unit's last V tile: zero its rows past the last key before P V reads them
+          // the unit's last V tile: P V reads its rows up to the next multiple of
+          // 16 past the last key; zero those past the last key first
           const int last_valid = u.kv_end - j * kTcKeys;
-          if (last_valid < kTcKeys) {
+          if (last_valid & 15) {
             const uint32_t iv = kv_unit + 2 * j + 1, slot = iv % kRing;
             if (!__all_sync(0xffffffffu, tc_wait(&bar->kv_full[slot], (iv / kRing) & 1, abort_flag,
                                                  p.err_flag))) {
               ok = false;
               break;
             }
-            const int nrow = kTcKeys - last_valid;
+            const int nrow = 16 - (last_valid & 15);
             for (int i = r; i < nrow * 8 * kHalves; i += kTcRows) {
               const int hf = i / (nrow * 8);
               const int rr = (i >> 3) % nrow;
@@ -652,21 +769,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const bool store = r < p.rows && q0 + qi < u.q_len;
       __nv_bfloat16* orow =
           p.out + ((int64_t)(u.q_start + q0 + qi) * p.hq + u.kvh * p.group + hh) * D;
+      uint32_t ov[D];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t ov[32];
-        tc::ld32(tO + c * 32, ov);
-        tc::wait_ld();
-        if (store) {
+      for (int c = 0; c < D / 32; ++c) tc::ld32(tO + c * 32, ov + c * 32);
+      tc::wait_ld();
+      if (store) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            uint4 v;
-            v.x = pack_bf16(__uint_as_float(ov[8 * k + 0]) * inv, __uint_as_float(ov[8 * k + 1]) * inv);
-            v.y = pack_bf16(__uint_as_float(ov[8 * k + 2]) * inv, __uint_as_float(ov[8 * k + 3]) * inv);
-            v.z = pack_bf16(__uint_as_float(ov[8 * k + 4]) * inv, __uint_as_float(ov[8 * k + 5]) * inv);
-            v.w = pack_bf16(__uint_as_float(ov[8 * k + 6]) * inv, __uint_as_float(ov[8 * k + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + c * 32 + k * 8) = v;
-          }
+        for (int k = 0; k < D / 8; ++k) {
+          uint4 v;
+          v.x = pack_bf16(__uint_as_float(ov[8 * k + 0]) * inv, __uint_as_float(ov[8 * k + 1]) * inv);
+          v.y = pack_bf16(__uint_as_float(ov[8 * k + 2]) * inv, __uint_as_float(ov[8 * k + 3]) * inv);
+          v.z = pack_bf16(__uint_as_float(ov[8 * k + 4]) * inv, __uint_as_float(ov[8 * k + 5]) * inv);
+          v.w = pack_bf16(__uint_as_float(ov[8 * k + 6]) * inv, __uint_as_float(ov[8 * k + 7]) * inv);
+          *reinterpret_cast<uint4*>(orow + k * 8) = v;
         }
       }
       // the next unit's first P V overwrites O_t: every lane's reads are done
