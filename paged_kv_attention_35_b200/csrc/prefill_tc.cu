@@ -28,16 +28,17 @@
 // ring streams across unit boundaries and the next unit's Q and first S
 // overlap the current unit's epilogue.
 //
-// Roles (10 warps):
+// Roles (11 warps):
 //   warp 8   producer: stages the unit's block-table entries in shared memory
 //            (one round trip), then Q tiles (one box per head-dim half) into
 //            two Q buffers and 128-key K and V tiles (one box per
 //            physical-block chunk, 128-byte swizzle) into a 5-slot ring.
-//   warp 9   MMA issuer (one thread): S_t(j) = Q_t K_j^T into the TMEM S
-//            columns (M=128, N=128, K=16 steps); O_t += P_t(j) V_j with P read
-//            from TMEM (TS form, B = V MN-major); per KV tile the order is
-//            S_A(j+1), P_A(j) V_j, S_B(j+1), P_B(j) V_j, so the tensor core
-//            works on one tile while the other tile's softmax runs.
+//   warps 9, 10   MMA issuers of tiles A and B (one thread each): S_t(j) =
+//            Q_t K_j^T into the TMEM S columns (M=128, N=128, K=16 steps);
+//            O_t += P_t(j) V_j with P read from TMEM (TS form, B = V MN-major);
+//            per tile S_t(j+1) goes before P_t(j) V_j, so the tensor core works
+//            on one tile while the other tile's softmax runs, and neither
+//            tile's P V waits for the other's softmax.
 //   warps 0-3 / 4-7   softmax of tile A / B, one thread per M row (TMEM lane):
 //            causal mask on the tiles that reach past a row's last key; online
 //            softmax in the log2 domain with a lazy rescale (the reference max
@@ -45,8 +46,9 @@
 //            of the exponentials is evaluated on the FMA pipe (exp2_poly2) so
 //            the MUFU unit is not the only one doing them; P as bf16 pairs
 //            written back over the S columns; epilogue O / l -> bf16 -> global.
-//            Tile A's warps also zero the last V tile's rows past the unit's
-//            last key before handing over that tile's P (stale pool rows may
+//            The warps of a tile that reads the unit's last V tile zero its rows
+//            past the unit's last key (up to the next multiple of 16: P V skips
+//            the 16-key steps beyond) before handing over P (stale pool rows may
 //            hold NaN, and 0 * NaN = NaN in P V).
 // TMEM: 512 columns: S (128, shared by the tiles in turn) | P_A (64) | P_B (64) |
 // O_A | O_B.  A tile's softmax releases the S columns as soon as S is in its
@@ -67,7 +69,9 @@ namespace pa {
 
 constexpr int kTcRows = 128;     // MMA M: packed (query, head) rows of a tile
 constexpr int kTcKeys = 128;     // keys per KV tile (MMA N of QK^T, K of PV)
-constexpr int kTcThreads = 320;  // 2 softmax warpgroups + producer warp + MMA warp
+constexpr int kTcThreads = 352;  // 2 softmax warpgroups + producer warp + 2 MMA warps
+// register budget of 12 warps (3 per SM sub-partition), which 11 warps then use
+constexpr int kTcBoundThreads = 384;
 constexpr int kTcHalf = kTcRows * 128;  // one 128-row x 64-element bf16 half (swizzled)
 constexpr int kRing = 5;         // K/V ring slots (K_j, V_j, K_j+1, ... in turn)
 // TMEM columns: S (shared by the two tiles in turn), P_A, P_B (bf16 pairs), O_A, O_B
@@ -280,6 +284,27 @@ __device__ __forceinline__ bool tc_wait_inline(uint64_t* bar, uint32_t parity,
   return res == 1;
 }
 
+// Waits until the shared counter reaches `target` (acquire), bounded like tc_wait.
+__device__ __forceinline__ bool tc_wait_count(uint32_t* ctr, uint32_t target,
+                                              volatile int* abort_flag, int32_t* err_flag) {
+  const uint32_t a = smem_u32(ctr);
+  uint64_t t0 = 0;
+  for (uint32_t i = 0;; ++i) {
+    uint32_t v;
+    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+    if ((int32_t)(v - target) >= 0) return true;
+    if (i == 0) t0 = globaltimer_ns();
+    if ((i & 255u) == 255u) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        raise_flag(err_flag, PA_FLAG_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
 // Packed / 3-input fp32 arithmetic of sm_100 (halves the softmax's issue slots).
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
@@ -344,7 +369,7 @@ struct Exp2Poly {
 
 constexpr int kBtCache = 256;    // block-table entries staged per unit
 constexpr int kUnitSlots = 4;    // unit descriptors the producer publishes ahead
-constexpr int kUnitReaders = 9;  // the MMA warp and the 8 softmax warps
+constexpr int kUnitReaders = 10; // the 2 MMA warps and the 8 softmax warps
 
 struct TcBars {
   uint64_t q_full[2];      // Q tile t landed
@@ -352,10 +377,14 @@ struct TcBars {
   uint64_t kv_full[kRing];
   uint64_t kv_empty[kRing];
   uint64_t s_full[2];      // S_t is in the S columns
-  uint64_t s_free;         // the S columns have been read into registers
+  // reads of tile t's S out of the S columns, counted per warp (4 per S): a
+  // monotonic count, not an mbarrier phase, because an issuer may wait for
+  // the other tile's next read before that tile's previous read is done,
+  // which a parity wait would take for complete
+  uint32_t s_reads[2];
   uint64_t p_full[2];      // P_t is in its TMEM columns (O_t rescaled if needed)
   uint64_t pv_done[2];     // the last P_t V issued is complete
-  uint64_t drain;
+  uint64_t drain[2];
   uint64_t unit_full[kUnitSlots];   // descriptor published (nt[0] == 0: no more units)
   uint64_t unit_empty[kUnitSlots];  // every reader has copied it
   TcUnit units[kUnitSlots];
@@ -383,7 +412,7 @@ __device__ __forceinline__ bool tc_take_unit(TcBars* bar, uint32_t k, int lane,
 }
 
 template <int D>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kTcBoundThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const PrefillTcParams p) {
   constexpr int kHalves = D / 64;
@@ -409,15 +438,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     mbar_init(&bar->q_empty[1], 1);
     for (int s = 0; s < kRing; ++s) {
       mbar_init(&bar->kv_full[s], 1);
-      mbar_init(&bar->kv_empty[s], 1);
+      mbar_init(&bar->kv_empty[s], 2);        // one commit per tile (both by A without B)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bar->s_full[t], 1);
       mbar_init(&bar->p_full[t], 4);
       mbar_init(&bar->pv_done[t], 1);
     }
-    mbar_init(&bar->drain, 1);
-    mbar_init(&bar->s_free, 4);
+    mbar_init(&bar->drain[0], 1);
+    mbar_init(&bar->drain[1], 1);
+    bar->s_reads[0] = 0;
+    bar->s_reads[1] = 0;
     for (int s = 0; s < kUnitSlots; ++s) {
       mbar_init(&bar->unit_full[s], 1);
       mbar_init(&bar->unit_empty[s], kUnitReaders);
@@ -439,7 +470,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     fence_proxy_async_smem();
   }
-  if (warp == 9) {
+  if (warp == 10) {
     tc::tmem_alloc(&bar->tmem, 512);
     tc::tmem_relinquish();
   }
@@ -527,29 +558,41 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // lane 0 is done with this unit's staged block table before it is overwritten
       if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    // The warp takes the unit descriptors; lane 0 issues every MMA.  Order
-    // per KV tile j:  S_A(j+1), P_A(j) V_j, S_B(j+1), P_B(j) V_j, where each
-    // S waits only until the previous S in the shared S columns has been
-    // read into registers, and each P V until that tile's P is in TMEM.
+  } else if (warp >= 9) {
+    // ------------------------------------------------------------ MMA issuers
+    // Warp 9 issues tile A's MMAs, warp 10 tile B's (lane 0; the warp takes
+    // the unit descriptors).  Per tile: S_t(j+1) before P_t(j) V_j, so the
+    // tile's next S is ready when its softmax finishes.  The S columns are
+    // used in one fixed order, A0 B0 A1 B1 ... (A alone once B has no more KV
+    // tiles), and every S waits until the previous S in that order has been
+    // read into registers; each P V waits only for its own tile's P.  (The
+    // protocol was checked by a model of all roles and of the asynchronous
+    // copies and MMAs under random schedules: no deadlock, no wait whose
+    // parity could alias another phase, and no unordered conflicting access
+    // other than the two tiles' identical zero writes to the last V tile.)
+    const int t = warp - 9;
     constexpr uint32_t idS = tc::idesc_bf16(kTcRows, kTcKeys, false, false);
     constexpr uint32_t idO = tc::idesc_bf16(kTcRows, D, false, true);
     // descriptors are built once; stepping K adds (byte offset / 16) to the
     // start-address field (no carry: shared addresses stay below 256 KB)
-    const uint64_t dQ0 = tc::sdesc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t dQ = tc::sdesc_sw128(smem_u32(sQ + t * kTile), 16, 1024);
     const uint64_t dK0 = tc::sdesc_sw128(smem_u32(sKV), 16, 1024);
     const uint64_t dV0 = tc::sdesc_sw128(smem_u32(sKV), kTcHalf, 1024);
-    uint32_t kv_i = 0, qc[2] = {0, 0}, pc[2] = {0, 0}, s_issued = 0;
+    uint32_t kv_i = 0, qc = 0, pc = 0;
+    // S groups of each tile in earlier units, and the last S of the previous
+    // unit (tile, index in that tile's sequence; tile -1: none yet)
+    uint32_t ra = 0, rb = 0;
+    int last_t = -1;
+    uint32_t last_i = 0;
     auto wait_kv = [&](uint32_t i) {
       return tc_wait(&bar->kv_full[i % kRing], (i / kRing) & 1, abort_flag, p.err_flag);
     };
-    // S_t = Q_t K^T into the shared S columns, once the previous S there has been read
-    auto issue_s = [&](int t, uint32_t kslot) {
-      if (s_issued > 0 && !tc_wait(&bar->s_free, (s_issued - 1) & 1, abort_flag, p.err_flag))
+    // S_t(j) = Q_t K_j^T into the shared S columns, once the S before it in
+    // the order (tile pt, pi-th S of that tile) has been read.
+    auto issue_s = [&](int pt, uint32_t pi, uint32_t kslot) {
+      if (pt >= 0 && !tc_wait_count(&bar->s_reads[pt], 4 * (pi + 1), abort_flag, p.err_flag))
         return false;
       tc::fence_after_sync();
-      const uint64_t dQ = dQ0 + (uint64_t)((t * kTile) >> 4);
       const uint64_t dK = dK0 + (uint64_t)((kslot * kTile) >> 4);
 #pragma unroll
       for (int ks = 0; ks < kSteps; ++ks) {
@@ -557,73 +600,79 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc::mma_ss(tmem + kTmemS, dQ + o, dK + o, idS, ks > 0);
       }
       tc::commit(&bar->s_full[t]);
-      ++s_issued;
-      return true;
-    };
-    // O_t += P_t V_j (the last tile: only the 16-key steps before kv_end)
-    auto issue_pv = [&](const TcUnit& u, int t, int j, uint32_t vslot) {
-      if (!tc_wait(&bar->p_full[t], pc[t]++ & 1, abort_flag, p.err_flag)) return false;
-      tc::fence_after_sync();
-      const uint64_t dV = dV0 + (uint64_t)((vslot * kTile) >> 4);
-      const int nks = j == u.nt[0] - 1 ? (u.kv_end - j * kTcKeys + 15) / 16 : kTcKeys / 16;
-#pragma unroll
-      for (int ks = 0; ks < kTcKeys / 16; ++ks)
-        if (ks < nks)
-          tc::mma_ts(tmem + kTmemO + kOCols * t, tmem + kTmemP + 64 * t + ks * 8,
-                     dV + (uint64_t)((ks * 2048) >> 4), idO, (j > 0 || ks > 0));
-      tc::commit(&bar->pv_done[t]);
       return true;
     };
     for (uint32_t k = 0;; ++k) {
       TcUnit u;
       bool ok = true;
       if (!tc_take_unit(bar, k, lane, abort_flag, p.err_flag, u, ok)) break;
-      if (lane == 0) {
-        const int n = u.nt[0], nb = u.nt[1];
-        for (int t = 0; t < 2 && ok; ++t)
-          if (u.nt[t] > 0) ok = tc_wait(&bar->q_full[t], qc[t]++ & 1, abort_flag, p.err_flag);
-        if (ok) ok = wait_kv(kv_i);                       // K_0
+      const int n = u.nt[0], nb = u.nt[1], nt = u.nt[t];
+      if (lane == 0 && nt > 0) {
+        // the S read before S_t(j) in the order A0 B0 A1 B1 ... A(nb) ... A(n-1)
+        auto pred_t = [&](int j) -> int {
+          return t == 1 ? 0 : (j == 0 ? last_t : (j - 1 < nb ? 1 : 0));
+        };
+        auto pred_i = [&](int j) -> uint32_t {
+          return t == 1 ? ra + j : (j == 0 ? last_i : (j - 1 < nb ? rb + j - 1 : ra + j - 1));
+        };
+        // K_j / V_j are released by one commit of each tile (tile A commits
+        // twice for the tiles B does not read)
+        auto release = [&](uint32_t slot, int j) {
+          tc::commit(&bar->kv_empty[slot]);
+          if (t == 0 && j >= nb) tc::commit(&bar->kv_empty[slot]);
+        };
+        ok = tc_wait(&bar->q_full[t], qc++ & 1, abort_flag, p.err_flag) && wait_kv(kv_i);
         if (ok) {
           tc::fence_after_sync();
-          ok = issue_s(0, kv_i % kRing);
-          if (ok && n == 1) tc::commit(&bar->q_empty[0]);
+          ok = issue_s(pred_t(0), pred_i(0), kv_i % kRing);
+          if (ok) {
+            if (nt == 1) tc::commit(&bar->q_empty[t]);
+            release(kv_i % kRing, 0);                       // K_0
+          }
         }
-        if (ok && nb > 0) {
-          ok = issue_s(1, kv_i % kRing);
-          if (ok && nb == 1) tc::commit(&bar->q_empty[1]);
-        }
-        if (ok) tc::commit(&bar->kv_empty[kv_i % kRing]);  // K_0 consumed
-        for (int j = 0; ok && j < n; ++j) {
+        for (int j = 0; ok && j < nt; ++j) {
           const uint32_t iv = kv_i + 2 * j + 1, vslot = iv % kRing;
           const uint32_t kn = iv + 1, kslot = kn % kRing;  // K_j+1
-          if (j + 1 < n) {
-            if (!wait_kv(kn)) { ok = false; break; }
-            if (!issue_s(0, kslot)) { ok = false; break; }
-            if (j + 2 == n) tc::commit(&bar->q_empty[0]);
+          if (j + 1 < nt) {
+            if (!wait_kv(kn) || !issue_s(pred_t(j + 1), pred_i(j + 1), kslot)) { ok = false; break; }
+            if (j + 2 == nt) tc::commit(&bar->q_empty[t]);
+            release(kslot, j + 1);
           }
-          // V_j's tail rows (last tile) are zeroed by tile A's softmax before it
-          // hands over P, so the V_j wait is the plain landing wait
-          if (!wait_kv(iv)) { ok = false; break; }
+          // O_t += P_t V_j (the last KV tile: only the 16-key steps before
+          // kv_end; both tiles' softmax warps zero V rows past the last key
+          // up to the next multiple of 16 before handing over P)
+          if (!wait_kv(iv) || !tc_wait(&bar->p_full[t], pc++ & 1, abort_flag, p.err_flag)) {
+            ok = false;
+            break;
+          }
           tc::fence_after_sync();
-          if (!issue_pv(u, 0, j, vslot)) { ok = false; break; }
-          if (j < nb) {
-            if (j + 1 < nb) {
-              if (!issue_s(1, kslot)) { ok = false; break; }
-              if (j + 2 == nb) tc::commit(&bar->q_empty[1]);
-            }
-            if (!issue_pv(u, 1, j, vslot)) { ok = false; break; }
-          }
-          tc::commit(&bar->kv_empty[vslot]);                 // V_j consumed
-          if (j + 1 < n) tc::commit(&bar->kv_empty[kslot]);  // K_j+1 consumed
+          const uint64_t dV = dV0 + (uint64_t)((vslot * kTile) >> 4);
+          const int nks = j == n - 1 ? (u.kv_end - j * kTcKeys + 15) / 16 : kTcKeys / 16;
+#pragma unroll
+          for (int ks = 0; ks < kTcKeys / 16; ++ks)
+            if (ks < nks)
+              tc::mma_ts(tmem + kTmemO + kOCols * t, tmem + kTmemP + 64 * t + ks * 8,
+                         dV + (uint64_t)((ks * 2048) >> 4), idO, (j > 0 || ks > 0));
+          tc::commit(&bar->pv_done[t]);
+          release(vslot, j);                                // V_j
         }
-        kv_i += 2 * n;
       }
+      if (nb == n) {
+        last_t = 1;
+        last_i = rb + nb - 1;
+      } else {
+        last_t = 0;
+        last_i = ra + n - 1;
+      }
+      ra += n;
+      rb += nb;
+      kv_i += 2 * n;
       if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
     }
     if (lane == 0) {
       // every issued MMA finishes before TMEM is released
-      tc::commit(&bar->drain);
-      mbar_wait(&bar->drain, 0);
+      tc::commit(&bar->drain[t]);
+      mbar_wait(&bar->drain[t], 0);
     }
     __syncwarp();
   } else {
@@ -662,7 +711,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // S is in registers: the next Q K^T may overwrite the S columns
         tc::fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar->s_free);
+        if (lane == 0) {
+          asm volatile("red.release.cta.shared::cta.add.u32 [%0], 1;" ::"r"(smem_u32(&bar->s_reads[t]))
+                       : "memory");
+        }
         const int t0 = j * kTcKeys;
         if (t0 + kTcKeys - 1 > limit) {            // tile reaches past the row's last key: mask
           const int lim = limit - t0;
@@ -718,9 +770,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc::fence_after_sync();
         tc::st32(tP, pk);
         tc::st32(tP + 32, pk + 32);
-        if (t == 0 && j == nt - 1) {
+        if (j == u.nt[0] - 1) {
           // the unit's last V tile: P V reads its rows up to the next multiple of
-          // 16 past the last key; zero those past the last key first
+          // 16 past the last key; zero those past the last key first (both
+          // tiles' warps write the same zeros, each before its own P V)
           const int last_valid = u.kv_end - j * kTcKeys;
           if (last_valid & 15) {
             const uint32_t iv = kv_unit + 2 * j + 1, slot = iv % kRing;
@@ -792,7 +845,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 10) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, 512);
   }
