@@ -706,7 +706,7 @@ __global__ void __launch_bounds__(kTcBoundThreads, 1)
         tc::fence_after_sync();
         float sv[kTcKeys];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tc::ld32(tS + c * 32, reinterpret_cast<uint32_t*>(sv) + c * 32);
+        tc::ld128(tS, reinterpret_cast<uint32_t*>(sv));
         tc::wait_ld();
         // S is in registers: the next Q K^T may overwrite the S columns
         tc::fence_before_sync();
@@ -721,15 +721,16 @@ __global__ void __launch_bounds__(kTcBoundThreads, 1)
 #pragma unroll
           for (int i = 0; i < kTcKeys; ++i) sv[i] = i <= lim ? sv[i] : -INFINITY;
         }
-        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float mx8[8];
 #pragma unroll
-        for (int i = 0; i < kTcKeys; i += 8) {
-          mx4[0] = max3f(mx4[0], sv[i + 0], sv[i + 1]);
-          mx4[1] = max3f(mx4[1], sv[i + 2], sv[i + 3]);
-          mx4[2] = max3f(mx4[2], sv[i + 4], sv[i + 5]);
-          mx4[3] = max3f(mx4[3], sv[i + 6], sv[i + 7]);
+        for (int c = 0; c < 8; ++c) mx8[c] = fmaxf(sv[2 * c], sv[2 * c + 1]);
+#pragma unroll
+        for (int i = 16; i < kTcKeys; i += 16) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) mx8[c] = max3f(mx8[c], sv[i + 2 * c], sv[i + 2 * c + 1]);
         }
-        const float mx = max3f(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * sl2;  // scale > 0
+        const float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]),
+                               fmaxf(mx8[6], mx8[7])) * sl2;  // scale > 0
         float alpha = 1.f;
         bool resc = false;
         if (m_ref == -INFINITY) {
@@ -742,7 +743,7 @@ __global__ void __launch_bounds__(kTcBoundThreads, 1)
         }
         const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
         const uint64_t sc2 = f32x2(sl2, sl2), nm2 = f32x2(neg_m, neg_m);
-        uint64_t rs2[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
+        uint64_t rs2[4] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f), f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
         // P as 64 bf16 pairs (kept in registers until the previous P_t V is done)
         uint32_t pk[kTcKeys / 2];
 #pragma unroll
@@ -757,7 +758,7 @@ __global__ void __launch_bounds__(kTcBoundThreads, 1)
               e0 = fast_exp2(x0);
               e1 = fast_exp2(x1);
             }
-            rs2[(i >> 1) & 1] = fadd2(rs2[(i >> 1) & 1], f32x2(e0, e1));
+            rs2[(i >> 1) & 3] = fadd2(rs2[(i >> 1) & 3], f32x2(e0, e1));
             pk[i >> 1] = pack_bf16(e0, e1);
           }
         }
@@ -768,8 +769,7 @@ __global__ void __launch_bounds__(kTcBoundThreads, 1)
           break;
         }
         tc::fence_after_sync();
-        tc::st32(tP, pk);
-        tc::st32(tP + 32, pk + 32);
+        tc::st64(tP, pk);
         if (j == u.nt[0] - 1) {
           // the unit's last V tile: P V reads its rows up to the next multiple of
           // 16 past the last key; zero those past the last key first (both
@@ -794,8 +794,8 @@ __global__ void __launch_bounds__(kTcBoundThreads, 1)
         }
         {
           float a0, a1, b0, b1;
-          f32x2_split(rs2[0], a0, a1);
-          f32x2_split(rs2[1], b0, b1);
+          f32x2_split(fadd2(rs2[0], rs2[2]), a0, a1);
+          f32x2_split(fadd2(rs2[1], rs2[3]), b0, b1);
           l += (a0 + a1) + (b0 + b1);
         }
         if (__any_sync(0xffffffffu, resc)) {
@@ -824,7 +824,12 @@ __global__ void __launch_bounds__(kTcBoundThreads, 1)
           p.out + ((int64_t)(u.q_start + q0 + qi) * p.hq + u.kvh * p.group + hh) * D;
       uint32_t ov[D];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) tc::ld32(tO + c * 32, ov + c * 32);
+      if (D == 128) {
+        tc::ld128(tO, ov);
+      } else {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) tc::ld32(tO + c * 32, ov + c * 32);
+      }
       tc::wait_ld();
       if (store) {
 #pragma unroll
