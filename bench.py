@@ -459,6 +459,7 @@ def secondary(torch, args, timer, pk):
         "total_q": int(w.md.total_q), "TFLOPs": round(tf, 1),
         "frac_bf16_peak": round(tf / pk["bf16_tflops"], 4),
         "frac_bf16_sustained": round(tf / pk["bf16_tflops_sustained"], 4),
+        "peak_source": pk["source"], "traffic": load_traffic("prefill_tc_kernel", "prefix_prefill"),
         "store_GBs": round(w.store_bytes() / (store_ms * 1e-3) / 1e9, 1)}
     del w
     torch.cuda.empty_cache()
