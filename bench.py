@@ -309,6 +309,17 @@ def bench_prefill(torch, steps, warmup, timer):
 
     segs = np.asarray(timer.time_steps(one, steps, marks=2))
     store_ms, attn_ms = float(segs[:, 0].mean()), float(segs[:, 1].mean())
+
+    # the same step as one launch: the store folded into the prefill (pa_prefill_store)
+    for _ in range(warmup):
+        w.fused_step()
+
+    def fused(ev):
+        ev[0].record(stream)
+        w.fused_step()
+        ev[1].record(stream)
+
+    w.fused_ms = float(np.asarray(timer.time_steps(fused, steps, marks=1))[:, 0].mean())
     return w, store_ms, attn_ms
 
 
@@ -460,7 +471,9 @@ def secondary(torch, args, timer, pk):
         "frac_bf16_peak": round(tf / pk["bf16_tflops"], 4),
         "frac_bf16_sustained": round(tf / pk["bf16_tflops_sustained"], 4),
         "peak_source": pk["source"], "traffic": load_traffic("prefill_tc_kernel", "prefix_prefill"),
-        "store_GBs": round(w.store_bytes() / (store_ms * 1e-3) / 1e9, 1)}
+        "store_GBs": round(w.store_bytes() / (store_ms * 1e-3) / 1e9, 1),
+        "fused_store_prefill_ms": round(w.fused_ms, 4),
+        "fused_TFLOPs": round(w.flops() / (w.fused_ms * 1e-3) / 1e12, 1)}
     del w
     torch.cuda.empty_cache()
     nbytes, ms = bench_store_large(torch, steps, warm, timer)
@@ -490,7 +503,8 @@ def only(args):
         w, store_ms, attn_ms = bench_prefill(torch, args.steps, args.warmup, timer)
         tf = w.flops() / (attn_ms * 1e-3) / 1e12
         res = {"workload": "prefix_prefill", "attn_ms": round(attn_ms, 4), "TFLOPs": round(tf, 1),
-               "frac_bf16_peak": round(tf / pk["bf16_tflops"], 4)}
+               "frac_bf16_peak": round(tf / pk["bf16_tflops"], 4), "store_ms": round(store_ms, 4),
+               "fused_store_prefill_ms": round(w.fused_ms, 4)}
     elif args.only == "decode":
         w = DecodeWorkload.from_spec(synth.WORKLOADS[args.workload],
                                      block_size=args.block_size or None).upload("cuda")

@@ -68,8 +68,8 @@ typedef enum { PA_BF16 = 0 } pa_dtype;
 #define PA_FLAG_BLOCK_OOB  2  /* block table entry outside [0, num_blocks)            */
 #define PA_FLAG_LEN_OOB    4  /* context/sequence length outside its declared bounds  */
 #define PA_FLAG_TIMEOUT    8  /* a bounded wait gave up                                */
-#define PA_FLAG_SLOT_MISMATCH 16  /* pa_decode_store: slot_mapping[i] is not the slot of
-                                     sequence i's newest position                    */
+#define PA_FLAG_SLOT_MISMATCH 16  /* pa_decode_store / pa_prefill_store: a slot_mapping
+                                     entry is not the block-table slot of its token  */
 
 typedef void* pa_stream_t;
 
@@ -251,6 +251,46 @@ PA_API pa_status pa_prefill_varlen(void* out, const void* q, int64_t q_token_str
                             int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
                             int32_t head_dim, int32_t block_size, int32_t num_blocks,
                             float scale, pa_dtype dtype, int32_t* err_flag, pa_stream_t stream);
+
+/*
+ * pa_prefill_store -- one prefill step's store_kvcache and prefill in one launch.
+ *
+ * Same pool contents and output as pa_store_kvcache(key, value,
+ * key_token_stride, value_token_stride, k_cache, v_cache, slot_mapping,
+ * cu_seqlens_q[num_seqs], ...) followed by pa_prefill_varlen(...) with the
+ * remaining arguments, when every new token's slot follows the block table:
+ * slot_mapping[cu_seqlens_q[i] + j] == block_tables[i][p / block_size] *
+ * block_size + p % block_size for p = k_len-q_len+j (the Block Manager's
+ * mapping, "From Sequences to Blocks", lnwmold.com item; the step's new K/V
+ * are written before attention reads them, "Preparation before computation",
+ * same item).  Attention reads the new keys and values straight from key /
+ * value and the cached prefix from the pool, so nothing waits for the store;
+ * each new (token, KV head) row is written to the pool once, by the CTA that
+ * computes that token's queries, during the same launch.  A TMA box of pool
+ * rows that holds both cached and new keys (a cached length that is not a
+ * multiple of min(block_size, 128)) has its new rows written before it is
+ * read.
+ *   key, value     device [total_q, Hkv, D] bf16, rows *_token_stride elements
+ *                  apart (>= Hkv*D, multiples of 8), 16-byte aligned
+ *   slot_mapping   device int32 [total_q]
+ * Tokens past cu_seqlens_q[num_seqs] belong to no sequence and are not stored.
+ * A slot past the pool writes nothing and sets PA_FLAG_SLOT_OOB; a slot
+ * (negative included) that breaks the mapping above sets
+ * PA_FLAG_SLOT_MISMATCH, and that sequence's output and the pool rows it
+ * touches are then unspecified.  Other arguments, limits and errors as
+ * pa_prefill_varlen.  Asynchronous on `stream`.
+ */
+PA_API pa_status pa_prefill_store(void* out, const void* q, int64_t q_token_stride,
+                                  const void* key, const void* value, int64_t key_token_stride,
+                                  int64_t value_token_stride, const int32_t* slot_mapping,
+                                  void* k_cache, void* v_cache, const int32_t* cu_seqlens_q,
+                                  const int32_t* cu_seqlens_k, int32_t max_seqlen_q,
+                                  int32_t max_seqlen_k, int32_t total_q,
+                                  const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                  int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                  int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                                  float scale, pa_dtype dtype, int32_t* err_flag,
+                                  pa_stream_t stream);
 
 /*
  * pa_watchdog_read -- copy (and clear) the device-global word where kernels

@@ -379,15 +379,17 @@ pa_status pa_decode_store(void* out, const void* q, int64_t q_token_stride, cons
                      dtype, err_flag, stream, &st);
 }
 
-pa_status pa_prefill_varlen(void* out, const void* q, int64_t q_token_stride, const void* k_cache,
-                            const void* v_cache, const int32_t* cu_seqlens_q,
-                            const int32_t* cu_seqlens_k, int32_t max_seqlen_q,
-                            int32_t max_seqlen_k, int32_t total_q, const int32_t* block_tables,
-                            int32_t max_blocks_per_seq, int32_t num_seqs, int32_t num_q_heads,
-                            int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
-                            int32_t num_blocks, float scale, pa_dtype dtype, int32_t* err_flag,
-                            pa_stream_t stream) {
-  t_last_error.clear();
+// Validation and launch shared by pa_prefill_varlen and pa_prefill_store
+// (fused store when a.slot_mapping is set).
+static pa_status prefill_entry(PrefillArgs& a, void* out, const void* q, int64_t q_token_stride,
+                               const void* k_cache, const void* v_cache,
+                               const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                               int32_t max_seqlen_q, int32_t max_seqlen_k, int32_t total_q,
+                               const int32_t* block_tables, int32_t max_blocks_per_seq,
+                               int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                               int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                               float scale, pa_dtype dtype, int32_t* err_flag,
+                               pa_stream_t stream) {
   pa_status s = check_common(k_cache, v_cache, num_q_heads, num_kv_heads, head_dim, block_size,
                              num_blocks, dtype);
   if (s != PA_OK) return s;
@@ -404,7 +406,14 @@ pa_status pa_prefill_varlen(void* out, const void* q, int64_t q_token_stride, co
   if (max_blocks_per_seq <= 0 || (int64_t)max_blocks_per_seq * block_size < max_seqlen_k)
     return fail(PA_ERR_INVALID_ARG, "max_blocks_per_seq*block_size < max_seqlen_k");
   if (!(scale > 0.f) || !std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale must be finite and > 0");
-  PrefillArgs a{};
+  if (a.slot_mapping) {
+    if (!a.key || !a.value) return fail(PA_ERR_INVALID_ARG, "key / value is NULL");
+    if (!aligned16(a.key) || !aligned16(a.value))
+      return fail(PA_ERR_INVALID_ARG, "key / value must be 16-byte aligned");
+    const int64_t row = (int64_t)num_kv_heads * head_dim;
+    if (a.key_stride < row || a.value_stride < row || a.key_stride % 8 || a.value_stride % 8)
+      return fail(PA_ERR_INVALID_ARG, "key/value token strides must be >= Hkv*D and multiples of 8");
+  }
   a.out = out; a.q = q; a.q_stride = q_token_stride; a.total_q = total_q;
   a.k_cache = k_cache; a.v_cache = v_cache; a.cu_q = cu_seqlens_q; a.cu_k = cu_seqlens_k;
   a.max_seqlen_q = max_seqlen_q; a.max_seqlen_k = max_seqlen_k;
@@ -413,6 +422,46 @@ pa_status pa_prefill_varlen(void* out, const void* q, int64_t q_token_stride, co
   a.block_size = block_size; a.num_blocks = num_blocks; a.scale = scale;
   a.err_flag = err_flag; a.stream = (cudaStream_t)stream;
   return launch_prefill(a);
+}
+
+pa_status pa_prefill_varlen(void* out, const void* q, int64_t q_token_stride, const void* k_cache,
+                            const void* v_cache, const int32_t* cu_seqlens_q,
+                            const int32_t* cu_seqlens_k, int32_t max_seqlen_q,
+                            int32_t max_seqlen_k, int32_t total_q, const int32_t* block_tables,
+                            int32_t max_blocks_per_seq, int32_t num_seqs, int32_t num_q_heads,
+                            int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                            int32_t num_blocks, float scale, pa_dtype dtype, int32_t* err_flag,
+                            pa_stream_t stream) {
+  t_last_error.clear();
+  PrefillArgs a{};
+  return prefill_entry(a, out, q, q_token_stride, k_cache, v_cache, cu_seqlens_q, cu_seqlens_k,
+                       max_seqlen_q, max_seqlen_k, total_q, block_tables, max_blocks_per_seq,
+                       num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                       scale, dtype, err_flag, stream);
+}
+
+pa_status pa_prefill_store(void* out, const void* q, int64_t q_token_stride, const void* key,
+                           const void* value, int64_t key_token_stride,
+                           int64_t value_token_stride, const int32_t* slot_mapping, void* k_cache,
+                           void* v_cache, const int32_t* cu_seqlens_q,
+                           const int32_t* cu_seqlens_k, int32_t max_seqlen_q,
+                           int32_t max_seqlen_k, int32_t total_q, const int32_t* block_tables,
+                           int32_t max_blocks_per_seq, int32_t num_seqs, int32_t num_q_heads,
+                           int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                           int32_t num_blocks, float scale, pa_dtype dtype, int32_t* err_flag,
+                           pa_stream_t stream) {
+  t_last_error.clear();
+  if (!slot_mapping) return fail(PA_ERR_INVALID_ARG, "slot_mapping is NULL");
+  PrefillArgs a{};
+  a.key = key;
+  a.value = value;
+  a.key_stride = key_token_stride;
+  a.value_stride = value_token_stride;
+  a.slot_mapping = slot_mapping;
+  return prefill_entry(a, out, q, q_token_stride, k_cache, v_cache, cu_seqlens_q, cu_seqlens_k,
+                       max_seqlen_q, max_seqlen_k, total_q, block_tables, max_blocks_per_seq,
+                       num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                       scale, dtype, err_flag, stream);
 }
 
 pa_status pa_watchdog_read(uint32_t* value) {

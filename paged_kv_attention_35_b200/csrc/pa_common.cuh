@@ -121,6 +121,12 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// The same for global memory: this thread's generic-proxy global writes
+// before later TMA reads of them.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 
 // ----------------------------------------------- programmatic dependent launch
 // Kernels are launched with programmatic stream serialization: a kernel may be

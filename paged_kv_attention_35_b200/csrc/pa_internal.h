@@ -106,6 +106,12 @@ struct PrefillArgs {
   float scale;
   int32_t* err_flag;
   cudaStream_t stream;
+  // fused store (slot_mapping != nullptr): the batch's new K/V rows, written
+  // to the pool by the same launch and read by attention from these arrays
+  const void* key = nullptr;
+  const void* value = nullptr;
+  int64_t key_stride = 0, value_stride = 0;   // elements between tokens
+  const int32_t* slot_mapping = nullptr;
 };
 
 pa_status launch_prefill(const PrefillArgs& a);

@@ -22,17 +22,20 @@
 // are listed from the most KV tiles to the fewest (bucket = tile A's KV tiles;
 // within a bucket by sequence, pair, KV head) and dealt out in a snake: CTA c
 // of G takes list positions c, 2G-1-c, 2G+c, 4G-1-c, ..., so the expensive
-// units go first and every CTA ends close to the mean.  Each role's warp walks
-// this list on its own (32 sequences per step, warp prefix sums; the bucket
-// of a pair follows in closed form from the sequence's lengths).  The K/V
+// units go first and every CTA ends close to the mean.  The producer warp
+// walks this list (32 sequences per step, warp prefix sums; the bucket of a
+// pair follows in closed form from the sequence's lengths) and hands each unit
+// to the other roles through a 4-slot queue in shared memory.  The K/V
 // ring streams across unit boundaries and the next unit's Q and first S
 // overlap the current unit's epilogue.
 //
-// Roles (11 warps):
+// Roles (11 warps; 12 with the fused store):
 //   warp 8   producer: stages the unit's block-table entries in shared memory
 //            (one round trip), then Q tiles (one box per head-dim half) into
 //            two Q buffers and 128-key K and V tiles (one box per
 //            physical-block chunk, 128-byte swizzle) into a 5-slot ring.
+//            With the fused store the new keys' boxes come from the step's
+//            new-row arrays instead of the pool.
 //   warps 9, 10   MMA issuers of tiles A and B (one thread each): S_t(j) =
 //            Q_t K_j^T into the TMEM S columns (M=128, N=128, K=16 steps);
 //            O_t += P_t(j) V_j with P read from TMEM (TS form, B = V MN-major);
@@ -42,14 +45,17 @@
 //   warps 0-3 / 4-7   softmax of tile A / B, one thread per M row (TMEM lane):
 //            causal mask on the tiles that reach past a row's last key; online
 //            softmax in the log2 domain with a lazy rescale (the reference max
-//            moves only when it grows by more than 8, i.e. 256x); a fixed share
-//            of the exponentials is evaluated on the FMA pipe (exp2_poly2) so
-//            the MUFU unit is not the only one doing them; P as bf16 pairs
-//            written back over the S columns; epilogue O / l -> bf16 -> global.
+//            moves only when it grows by more than 8, i.e. 256x); exponentials
+//            on the MUFU unit (a polynomial on the FMA pipe, Exp2Poly, can take
+//            a share of them: kEmuPairs); P as bf16 pairs in the tile's TMEM
+//            P columns; epilogue O / l -> bf16 -> global.
 //            The warps of a tile that reads the unit's last V tile zero its rows
 //            past the unit's last key (up to the next multiple of 16: P V skips
 //            the 16-key steps beyond) before handing over P (stale pool rows may
 //            hold NaN, and 0 * NaN = NaN in P V).
+//   warp 11  (fused store only) writes the step's new K/V rows to their pool
+//            slots: the tokens of each of the CTA's units, walking the unit
+//            list on its own, since attention does not read those rows back.
 // TMEM: 512 columns: S (128, shared by the tiles in turn) | P_A (64) | P_B (64) |
 // O_A | O_B.  A tile's softmax releases the S columns as soon as S is in its
 // registers, so the next Q K^T overlaps the exponentials instead of waiting
@@ -70,7 +76,8 @@ namespace pa {
 constexpr int kTcRows = 128;     // MMA M: packed (query, head) rows of a tile
 constexpr int kTcKeys = 128;     // keys per KV tile (MMA N of QK^T, K of PV)
 constexpr int kTcThreads = 352;  // 2 softmax warpgroups + producer warp + 2 MMA warps
-// register budget of 12 warps (3 per SM sub-partition), which 11 warps then use
+// with the fused store, warp 11 writes the batch's new K/V rows to the pool;
+// the register budget is that of 12 warps (3 per SM sub-partition) either way
 constexpr int kTcBoundThreads = 384;
 constexpr int kTcHalf = kTcRows * 128;  // one 128-row x 64-element bf16 half (swizzled)
 constexpr int kRing = 5;         // K/V ring slots (K_j, V_j, K_j+1, ... in turn)
@@ -95,6 +102,13 @@ struct PrefillTcParams {
   int buckets;                     // KV tiles of the longest tile: ceil(max_seqlen_k / 128)
   float scale_log2;
   int32_t* err_flag;
+  // fused store (slots != nullptr): new K/V rows [total_q, hkv, D] and their pool slots
+  const int32_t* slots;
+  const uint4* new_k;
+  const uint4* new_v;
+  int64_t new_k_stride16, new_v_stride16;   // 16-byte chunks between tokens
+  uint4* kc;
+  uint4* vc;
 };
 
 // One work unit: tiles A (t = 0) and B (t = 1) of a (sequence, KV head).
@@ -367,6 +381,73 @@ struct Exp2Poly {
   }
 };
 
+// Streaming 16-byte global accesses that leave L1 alone (the fused store
+// touches each byte once).
+__device__ __forceinline__ uint4 ld_stream16(const uint4* a) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(a));
+  return v;
+}
+__device__ __forceinline__ void st_stream16(uint4* a, uint4 v) {
+  asm volatile("st.global.L1::no_allocate.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(a), "r"(v.x),
+               "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// Fused store: copies the new K/V rows of a sequence's new tokens [r0, r1)
+// (token r is key position cached + r) for KV head kvh to their pool slots.
+// Per group of 32 tokens, lane j reads token j's slot (and, with `check`, its
+// block-table slot: a slot that differs raises PA_FLAG_SLOT_MISMATCH, one past
+// the pool PA_FLAG_SLOT_OOB) in one coalesced load; then the rows are copied
+// in 16-byte chunks spread over the warp, kBatch loads in flight per lane.
+// Negative and out-of-pool slots write nothing.
+template <int D>
+__device__ __forceinline__ void tc_store_rows(const PrefillTcParams& p, int q_start, int cached,
+                                              const int32_t* bt, int kvh, int r0, int r1, int lane,
+                                              bool check) {
+  constexpr int C = D / 8;             // chunks of one K or V row
+  constexpr int kPer = 2 * C;          // chunks of a token: K, then V
+  constexpr int kTok = 32 / kPer;      // tokens one warp-wide access covers
+  constexpr int kBatch = 8;
+  const int c = lane % kPer, ch = c % C;
+  const bool isv = c >= C;
+  const uint4* src = (isv ? p.new_v : p.new_k) + kvh * C + ch;
+  const int64_t sstride = isv ? p.new_v_stride16 : p.new_k_stride16;
+  uint4* pool = (isv ? p.vc : p.kc) + kvh * C + ch;
+  for (int g = r0; g < r1; g += 32) {
+    const int n = min(32, r1 - g);
+    int slot = -1;
+    if (lane < n) {
+      slot = __ldg(p.slots + q_start + g + lane);
+      if (check) {
+        const int k = cached + g + lane;
+        const int bid = __ldg(bt + (k >> p.log2_bs));
+        if (slot >= p.num_slots)
+          raise_flag(p.err_flag, PA_FLAG_SLOT_OOB);
+        else if (bid >= 0 && bid < p.num_blocks &&
+                 slot != bid * p.block_size + (k & (p.block_size - 1)))
+          raise_flag(p.err_flag, PA_FLAG_SLOT_MISMATCH);
+      }
+    }
+    for (int t0 = 0; t0 < n; t0 += kBatch * kTok) {
+      uint4 v[kBatch];
+      int sl[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int t = t0 + u * kTok + lane / kPer;       // token within the group (< 32 + kBatch)
+        sl[u] = __shfl_sync(0xffffffffu, slot, t & 31);
+        if (t >= n) sl[u] = -1;
+        if (sl[u] >= 0) v[u] = ld_stream16(src + (int64_t)(q_start + g + t) * sstride);
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+        if (sl[u] >= 0 && sl[u] < p.num_slots) st_stream16(pool + (int64_t)sl[u] * p.hkv * C, v[u]);
+    }
+  }
+}
+
 constexpr int kBtCache = 256;    // block-table entries staged per unit
 constexpr int kUnitSlots = 4;    // unit descriptors the producer publishes ahead
 constexpr int kUnitReaders = 10; // the 2 MMA warps and the 8 softmax warps
@@ -414,7 +495,8 @@ __device__ __forceinline__ bool tc_take_unit(TcBars* bar, uint32_t k, int lane,
 template <int D>
 __global__ void __launch_bounds__(kTcBoundThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmV, const PrefillTcParams p) {
+                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmNK,
+                      const __grid_constant__ CUtensorMap tmNV, const PrefillTcParams p) {
   constexpr int kHalves = D / 64;
   constexpr uint32_t kOCols = D;               // TMEM columns of one O accumulator
   constexpr int kTile = kHalves * kTcHalf;     // one Q, K or V tile
@@ -458,12 +540,16 @@ __global__ void __launch_bounds__(kTcBoundThreads, 1)
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    if (p.slots) {
+      tma_prefetch_desc(&tmNK);
+      tma_prefetch_desc(&tmNV);
+    }
   }
   // rows >= p.rows of the Q buffers are never written by TMA: zero them once so
   // the padding rows of S stay finite
   {
     const int pad = kTcRows - p.rows;
-    for (int i = threadIdx.x; i < 2 * kHalves * pad * 8; i += kTcThreads) {
+    for (int i = threadIdx.x; i < 2 * kHalves * pad * 8; i += blockDim.x) {
       const int chunk = i & 7, rr = (i >> 3) % pad, hb = (i >> 3) / pad;   // hb = buffer * kHalves + half
       *reinterpret_cast<uint4*>(sQ + hb * kTcHalf + (p.rows + rr) * 128 + chunk * 16) =
           make_uint4(0, 0, 0, 0);
@@ -505,6 +591,16 @@ __global__ void __launch_bounds__(kTcBoundThreads, 1)
       const int32_t* bt = p.block_tables + (int64_t)u.seq * p.max_blocks;
       const int nblk = min((u.kv_end + p.block_size - 1) >> p.log2_bs, kBtCache);
       for (int i = lane; i < nblk; i += 32) bar->bt[i] = __ldg(bt + i);
+      // fused store: keys from the cached length on are read from the new-row
+      // arrays, box by box; a box that holds both cached and new keys (cached
+      // length not a multiple of the box) is read from the pool, so its new
+      // rows are written there first (the store warp writes the same values)
+      const bool fused = p.slots != nullptr;
+      const int split = fused ? min(u.kv_end, (u.cached + box - 1) / box * box) : 0;
+      if (fused && split > u.cached) {
+        tc_store_rows<D>(p, u.q_start, u.cached, bt, u.kvh, 0, split - u.cached, lane, false);
+        fence_proxy_async_global();
+      }
       __syncwarp();
       bool ok = true;
       if (lane == 0) {
@@ -528,6 +624,10 @@ __global__ void __launch_bounds__(kTcBoundThreads, 1)
           int rows[kTcKeys / 16];
           for (int b = 0; b < nbox; ++b) {
             const int t = t0 + b * box;
+            if (fused && t >= split) {                 // new keys: token rows of the arrays
+              rows[b] = -1 - (u.q_start + t - u.cached);
+              continue;
+            }
             const int lb = t >> p.log2_bs;
             const int bid = lb < kBtCache ? bar->bt[lb] : __ldg(bt + lb);
             if (bid < 0 || bid >= p.num_blocks) {
@@ -544,13 +644,15 @@ __global__ void __launch_bounds__(kTcBoundThreads, 1)
               ok = false;
               break;
             }
-            const CUtensorMap* map = kv ? &tmV : &tmK;
             mbar_arrive_expect_tx(&bar->kv_full[slot], bytes);
             for (int b = 0; b < nbox; ++b) {
               uint8_t* dst = sKV + slot * kTile + b * box * 128;
+              const bool arr = rows[b] < 0;
+              const CUtensorMap* map = arr ? (kv ? &tmNV : &tmNK) : (kv ? &tmV : &tmK);
+              const int row = arr ? -1 - rows[b] : rows[b];
 #pragma unroll
               for (int hf = 0; hf < kHalves; ++hf)
-                tma_load_3d(dst + hf * kTcHalf, map, &bar->kv_full[slot], hf * 64, u.kvh, rows[b]);
+                tma_load_3d(dst + hf * kTcHalf, map, &bar->kv_full[slot], hf * 64, u.kvh, row);
             }
           }
         }
@@ -558,7 +660,7 @@ __global__ void __launch_bounds__(kTcBoundThreads, 1)
       // lane 0 is done with this unit's staged block table before it is overwritten
       if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
     }
-  } else if (warp >= 9) {
+  } else if (warp == 9 || warp == 10) {
     // ------------------------------------------------------------ MMA issuers
     // Warp 9 issues tile A's MMAs, warp 10 tile B's (lane 0; the warp takes
     // the unit descriptors).  Per tile: S_t(j+1) before P_t(j) V_j, so the
@@ -675,6 +777,25 @@ __global__ void __launch_bounds__(kTcBoundThreads, 1)
       mbar_wait(&bar->drain[t], 0);
     }
     __syncwarp();
+  } else if (warp == 11) {
+    // ------------------------------------------------------------ fused store
+    // (present only with the fused store) each unit's own tokens, tile B's
+    // first query to tile A's last, for the unit's KV head: every (token, KV
+    // head) of the batch belongs to exactly one unit, so each new row is
+    // written once.  Attention reads the new rows from the arrays, so nothing
+    // waits for these writes: this warp walks the CTA's unit list on its own
+    // and runs ahead of the other roles instead of taking the published units.
+    TcWalk walk;
+    walk.init(p);
+    for (int k = 0;; ++k) {
+      TcUnit u;
+      if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;   // warp-uniform: the walk shuffles
+      if (!walk.find(p, tc_position(k), lane, false, u)) break;
+      const int r0 = u.nt[1] > 0 ? u.q0[1] : u.q0[0];
+      const int r1 = min(u.q_len, u.q0[0] + p.qpt);
+      tc_store_rows<D>(p, u.q_start, u.cached, p.block_tables + (int64_t)u.seq * p.max_blocks,
+                       u.kvh, r0, r1, lane, true);
+    }
   } else {
     // ------------------------------------------------------------ softmax (warpgroup t = tile)
     const int t = warp >> 2;                       // 0: tile A, 1: tile B
@@ -705,7 +826,6 @@ __global__ void __launch_bounds__(kTcBoundThreads, 1)
         }
         tc::fence_after_sync();
         float sv[kTcKeys];
-#pragma unroll
         tc::ld128(tS, reinterpret_cast<uint32_t*>(sv));
         tc::wait_ld();
         // S is in registers: the next Q K^T may overwrite the S columns
@@ -823,7 +943,6 @@ __global__ void __launch_bounds__(kTcBoundThreads, 1)
       __nv_bfloat16* orow =
           p.out + ((int64_t)(u.q_start + q0 + qi) * p.hq + u.kvh * p.group + hh) * D;
       uint32_t ov[D];
-#pragma unroll
       if (D == 128) {
         tc::ld128(tO, ov);
       } else {
@@ -871,6 +990,14 @@ static pa_status launch_prefill_d(const PrefillArgs& a) {
   if (s != PA_OK) return s;
   s = get_tensor_map(&mv, a.v_cache, slots, a.hkv, a.d, (int64_t)a.hkv * a.d, box);
   if (s != PA_OK) return s;
+  const bool fused = a.slot_mapping != nullptr;
+  CUtensorMap mnk = mk, mnv = mv;                // the new-row arrays (fused store only)
+  if (fused) {
+    s = get_tensor_map(&mnk, a.key, a.total_q, a.hkv, a.d, a.key_stride, box);
+    if (s != PA_OK) return s;
+    s = get_tensor_map(&mnv, a.value, a.total_q, a.hkv, a.d, a.value_stride, box);
+    if (s != PA_OK) return s;
+  }
   PrefillTcParams prm{};
   prm.out = static_cast<__nv_bfloat16*>(a.out);
   prm.cu_q = a.cu_q;
@@ -896,6 +1023,15 @@ static pa_status launch_prefill_d(const PrefillArgs& a) {
   const int64_t max_units = max_pairs * a.num_seqs * a.hkv;
   prm.scale_log2 = a.scale * 1.4426950408889634f;
   prm.err_flag = a.err_flag;
+  if (fused) {
+    prm.slots = a.slot_mapping;
+    prm.new_k = static_cast<const uint4*>(a.key);
+    prm.new_v = static_cast<const uint4*>(a.value);
+    prm.new_k_stride16 = a.key_stride / 8;
+    prm.new_v_stride16 = a.value_stride / 8;
+    prm.kc = static_cast<uint4*>(const_cast<void*>(a.k_cache));
+    prm.vc = static_cast<uint4*>(const_cast<void*>(a.v_cache));
+  }
   // at least 120 KB so that two CTAs never share an SM (each allocates all 512
   // TMEM columns)
   static_assert((2 + kRing) * (size_t)kTile + 1024 + sizeof(TcBars) <= 232448,
@@ -905,8 +1041,9 @@ static pa_status launch_prefill_d(const PrefillArgs& a) {
   s = ensure_smem_attr((const void*)prefill_tc_kernel<D>, (int)smem, "prefill smem attribute");
   if (s != PA_OK) return s;
   const int64_t ctas = max_units < device_sm_count() ? max_units : device_sm_count();
-  cudaError_t e = launch_pdl(prefill_tc_kernel<D>, dim3((unsigned)ctas), dim3(kTcThreads), smem,
-                             a.stream, mq, mk, mv, prm);
+  cudaError_t e = launch_pdl(prefill_tc_kernel<D>, dim3((unsigned)ctas),
+                             dim3(fused ? kTcThreads + 32 : kTcThreads), smem, a.stream, mq, mk,
+                             mv, mnk, mnv, prm);
   if (e != cudaSuccess) {
     forget_smem_attr((const void*)prefill_tc_kernel<D>);
     return cuda_fail(e, "prefill launch");

@@ -49,6 +49,9 @@ SIGNATURES = {
                            _i32, _f32, _i32, ctypes.c_int, _p, _p], ctypes.c_int),
     "pa_prefill_varlen": ([_p, _p, _i64, _p, _p, _p, _p, _i32, _i32, _i32, _p, _i32, _i32, _i32, _i32,
                            _i32, _i32, _i32, _f32, ctypes.c_int, _p, _p], ctypes.c_int),
+    "pa_prefill_store": ([_p, _p, _i64, _p, _p, _i64, _i64, _p, _p, _p, _p, _p, _i32, _i32, _i32,
+                          _p, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32, ctypes.c_int, _p, _p],
+                         ctypes.c_int),
     "pa_watchdog_read": ([ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
     "pa_selftest_wait_timeout": ([_p, ctypes.c_uint32, _p, _p], ctypes.c_int),
 }
@@ -246,6 +249,39 @@ def prefill_varlen(q, k_cache, v_cache, cu_seqlens_q, cu_seqlens_k, max_seqlen_q
                                   int(max_seqlen_q), int(max_seqlen_k), total_q, _ptr(block_tables),
                                   block_tables.shape[1], num_seqs, hq, hkv, d, bs, nb, float(scale),
                                   PA_BF16, _ptr(err_flag), _stream()), "pa_prefill_varlen")
+    return out
+
+
+def prefill_store(q, key, value, k_cache, v_cache, slot_mapping, cu_seqlens_q, cu_seqlens_k,
+                  max_seqlen_q, max_seqlen_k, block_tables, scale=None, out=None, err_flag=None):
+    """One prefill step's ``store_kvcache`` and ``prefill_varlen`` in one launch
+    (``pa_prefill_store``): key/value [total_q, Hkv, D] rows go to ``slot_mapping`` while
+    q [total_q, Hq, D] attends over the cached prefix in the pool and the new rows -> out."""
+    _need_cuda(q=q, key=key, value=value, k_cache=k_cache, v_cache=v_cache,
+               slot_mapping=slot_mapping, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k,
+               block_tables=block_tables, out=out, err_flag=err_flag)
+    _need_bf16(q=q, key=key, value=value, k_cache=k_cache, v_cache=v_cache)
+    _need_i32(slot_mapping=slot_mapping, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k,
+              block_tables=block_tables)
+    nb, bs, hkv, d = k_cache.shape
+    total_q, hq, dq = q.shape
+    if dq != d:
+        raise ValueError("q head_dim differs from the pool's")
+    if (key.shape[0] != total_q or value.shape[0] != total_q or slot_mapping.numel() != total_q
+            or tuple(key.shape[1:]) != (hkv, d) or tuple(value.shape[1:]) != (hkv, d)):
+        raise ValueError("prefill_store takes one key/value row and slot per query token")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((total_q, hq, d), dtype=torch.bfloat16, device=q.device)
+    num_seqs = cu_seqlens_q.numel() - 1
+    _check(_lib.pa_prefill_store(_ptr(out), _ptr(q), _token_stride(q, "q"), _ptr(key), _ptr(value),
+                                 _token_stride(key, "key"), _token_stride(value, "value"),
+                                 _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache),
+                                 _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), int(max_seqlen_q),
+                                 int(max_seqlen_k), total_q, _ptr(block_tables),
+                                 block_tables.shape[1], num_seqs, hq, hkv, d, bs, nb, float(scale),
+                                 PA_BF16, _ptr(err_flag), _stream()), "pa_prefill_store")
     return out
 
 

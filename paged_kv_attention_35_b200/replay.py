@@ -10,8 +10,8 @@ seeded random id.
 
 One step: ``Scheduler.schedule()`` -> ``prepare_prefill`` / ``prepare_decode``
 -> one pinned host->device copy of the packed int32 metadata -> for every
-layer: ``store_kvcache`` of the step's new K/V rows into that layer's pool
-and ``prefill_varlen``, or both fused in ``decode_store``, into a scratch output -> postprocess
+layer: the store of the step's new K/V rows into that layer's pool and the
+attention, one launch (``prefill_store`` / ``decode_store``), into a scratch output -> postprocess
 (append tokens, finish, free).  All launches go to the current stream; the
 host runs ahead of the GPU except where it reuses a pinned staging buffer.
 
@@ -288,9 +288,10 @@ class Replay:
             r = self.ring_index(self.step_idx, layer)
             kc, vc = self.k_pools[layer], self.v_pools[layer]
             if is_prefill:
-                ops.store_kvcache(self.k_ring[r, :n], self.v_ring[r, :n], kc, vc, slots)
-                ops.prefill_varlen(self.q_ring[r, :n], kc, vc, cu_q, cu_k, md.max_seqlen_q,
-                                   md.max_seqlen_k, bt, out=out)
+                # the step's store fused into the prefill launch (pa_prefill_store)
+                ops.prefill_store(self.q_ring[r, :n], self.k_ring[r, :n], self.v_ring[r, :n], kc,
+                                  vc, slots, cu_q, cu_k, md.max_seqlen_q, md.max_seqlen_k, bt,
+                                  out=out)
             else:
                 # the step's store fused into the decode launch (pa_decode_store)
                 ops.decode_store(self.q_ring[r, :n], self.k_ring[r, :n], self.v_ring[r, :n], kc, vc,
@@ -306,8 +307,8 @@ class Replay:
         else:
             split = not is_prefill and ops.decode_workspace_size(
                 n, c.num_q_heads, c.num_kv_heads, c.head_dim, md.max_context_len) > 0
-        # prefill: store + attention; decode: the fused store + decode, and the merge
-        self.stats["launches"] += c.num_layers * (2 if is_prefill else (2 if split else 1))
+        # prefill: the fused store + attention; decode: the fused store + decode, and the merge
+        self.stats["launches"] += c.num_layers * (1 if is_prefill else (2 if split else 1))
         ev1 = torch.cuda.Event(enable_timing=True)
         ev1.record()
         self.step_events.append((ev0, ev1))

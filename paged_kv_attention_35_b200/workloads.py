@@ -198,6 +198,13 @@ class PrefixPrefillWorkload:
         self.store(err_flag)
         return self.attend(err_flag)
 
+    def fused_step(self, err_flag=None):
+        """The same step in one launch: the store folded into the prefill (``prefill_store``)."""
+        from . import ops
+        return ops.prefill_store(self.d_q, self.d_new_k, self.d_new_v, self.kc, self.vc,
+                                 self.d_slots, self.d_cu_q, self.d_cu_k, self.md.max_seqlen_q,
+                                 self.md.max_seqlen_k, self.d_bt, out=self.d_out, err_flag=err_flag)
+
     def flops(self) -> int:
         """Causal algorithmic FLOPs: 4*D*Hq per visible (query, key) pair."""
         total = 0
