@@ -735,28 +735,64 @@ __global__ void __launch_bounds__(kTcBoundThreads, 1)
         for (int j = 0; ok && j < nt; ++j) {
           const uint32_t iv = kv_i + 2 * j + 1, vslot = iv % kRing;
           const uint32_t kn = iv + 1, kslot = kn % kRing;  // K_j+1
-          if (j + 1 < nt) {
-            if (!wait_kv(kn) || !issue_s(pred_t(j + 1), pred_i(j + 1), kslot)) { ok = false; break; }
-            if (j + 2 == nt) tc::commit(&bar->q_empty[t]);
-            release(kslot, j + 1);
-          }
-          // O_t += P_t V_j (the last KV tile: only the 16-key steps before
-          // kv_end; both tiles' softmax warps zero V rows past the last key
-          // up to the next multiple of 16 before handing over P)
-          if (!wait_kv(iv) || !tc_wait(&bar->p_full[t], pc++ & 1, abort_flag, p.err_flag)) {
-            ok = false;
-            break;
-          }
-          tc::fence_after_sync();
-          const uint64_t dV = dV0 + (uint64_t)((vslot * kTile) >> 4);
-          const int nks = j == n - 1 ? (u.kv_end - j * kTcKeys + 15) / 16 : kTcKeys / 16;
+          // S_t(j+1) and P_t(j) V_j in whichever order their inputs become
+          // ready: S_t(j+1) waits for the other tile's read of the S columns,
+          // and a P V held behind that wait would hold up this tile's
+          // softmax, which rewrites P_t only after P_t V has completed
+          bool s_todo = j + 1 < nt, pv_todo = true;
+          const int spt = s_todo ? pred_t(j + 1) : -1;
+          const uint32_t spi = s_todo ? pred_i(j + 1) : 0;
+          uint64_t w0 = 0;
+          for (uint32_t spin = 0; s_todo || pv_todo; ++spin) {
+            bool progressed = false;
+            if (s_todo && mbar_test_wait(&bar->kv_full[kn % kRing], (kn / kRing) & 1)) {
+              uint32_t v = 4 * (spi + 1);
+              if (spt >= 0)
+                asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];"
+                             : "=r"(v) : "r"(smem_u32(&bar->s_reads[spt])) : "memory");
+              if ((int32_t)(v - 4 * (spi + 1)) >= 0) {
+                issue_s(-1, 0, kslot);                    // (its predecessor was read: no wait)
+                if (j + 2 == nt) tc::commit(&bar->q_empty[t]);
+                release(kslot, j + 1);
+                s_todo = false;
+                progressed = true;
+              }
+            }
+            if (pv_todo && mbar_test_wait(&bar->kv_full[vslot], (iv / kRing) & 1) &&
+                mbar_test_wait(&bar->p_full[t], pc & 1)) {
+              ++pc;
+              // O_t += P_t V_j (the last KV tile: only the 16-key steps before
+              // kv_end; both tiles' softmax warps zero V rows past the last key
+              // up to the next multiple of 16 before handing over P)
+              tc::fence_after_sync();
+              const uint64_t dV = dV0 + (uint64_t)((vslot * kTile) >> 4);
+              const int nks = j == n - 1 ? (u.kv_end - j * kTcKeys + 15) / 16 : kTcKeys / 16;
 #pragma unroll
-          for (int ks = 0; ks < kTcKeys / 16; ++ks)
-            if (ks < nks)
-              tc::mma_ts(tmem + kTmemO + kOCols * t, tmem + kTmemP + 64 * t + ks * 8,
-                         dV + (uint64_t)((ks * 2048) >> 4), idO, (j > 0 || ks > 0));
-          tc::commit(&bar->pv_done[t]);
-          release(vslot, j);                                // V_j
+              for (int ks = 0; ks < kTcKeys / 16; ++ks)
+                if (ks < nks)
+                  tc::mma_ts(tmem + kTmemO + kOCols * t, tmem + kTmemP + 64 * t + ks * 8,
+                             dV + (uint64_t)((ks * 2048) >> 4), idO, (j > 0 || ks > 0));
+              tc::commit(&bar->pv_done[t]);
+              release(vslot, j);                            // V_j
+              pv_todo = false;
+              progressed = true;
+            }
+            if (!progressed && (spin & 255u) == 255u) {
+              if (*abort_flag) {
+                ok = false;
+                break;
+              }
+              const uint64_t now = globaltimer_ns();
+              if (w0 == 0) {
+                w0 = now;
+              } else if (now - w0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                raise_flag(p.err_flag, PA_FLAG_TIMEOUT);
+                ok = false;
+                break;
+              }
+            }
+          }
         }
       }
       if (nb == n) {
