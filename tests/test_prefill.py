@@ -131,3 +131,10 @@ def test_prefill_many_sequences(cuda_device):
     out = c.run_gpu()
     seqs = list(range(0, 300, 7))
     compare(out[torch.from_numpy(c.rows_of(seqs)).cuda()], c.oracle_prefill(seqs), "many seqs")
+
+
+def test_prefill_block_table_past_staged_entries(cuda_device):
+    """Block 16 with 5,000-token sequences: a unit's keys span up to 313 blocks, past the 256
+    block-table entries the producer stages in shared memory (the rest are read directly)."""
+    c = PrefillCase([1000, 3], [4000, 4997], hq=8, hkv=2, d=64, bs=16, seed=41)
+    compare(c.run_gpu(), c.oracle_prefill(), "prefill past staged block-table entries")

@@ -200,3 +200,15 @@ def test_fused_slot_checks(cuda_device):
     # every other row is in place, the out-of-pool row went nowhere
     ref = _two_launch(c, key, value, oob, q, cu_q, cu_k, bt)
     assert torch.equal(_bits(got[1]), _bits(ref[1])) and torch.equal(_bits(got[2]), _bits(ref[2]))
+
+
+def test_fused_block_table_past_staged_entries(cuda_device):
+    """The fused store at block 16 with 5,000-token sequences (block tables longer than the
+    256 entries staged per unit; a cached length of 3 leaves a box of cached and new keys)."""
+    c = PrefillCase([1000, 3], [4000, 4997], hq=8, hkv=2, d=64, bs=16, seed=43)
+    key, value, slots = _new_rows(c)
+    q, cu_q, cu_k, bt = _inputs(c)
+    ref = _two_launch(c, key, value, slots, q, cu_q, cu_k, bt)
+    got = _fused(c, key, value, slots, q, cu_q, cu_k, bt)
+    assert got[3] == 0
+    _check_same(got, ref, "block 16, 5000 tokens")
