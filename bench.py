@@ -498,6 +498,73 @@ def ours(args):
         dist.destroy_process_group()
 
 
+def library_comparison(torch, steps, warmup, timer):
+    """FlashAttention-2 (`flash_attn`, installed in the image: the attention library the
+    pages' engine calls) on the same inputs, as a black-box comparison, never as the oracle:
+    paged decode (`flash_attn_with_kvcache` with the block tables) on the 7B-GQA and Qwen3
+    decode workloads, and paged varlen prefill (`flash_attn_varlen_func` with the block
+    tables) on the prefix-cached prefill, each beside this library's kernel on the same
+    buffers, timed the same way (events, L2 flushed before every launch)."""
+    from paged_kv_attention_35_b200 import ops, synth
+    from paged_kv_attention_35_b200.workloads import DecodeWorkload, PrefixPrefillWorkload
+    try:
+        from flash_attn import flash_attn_with_kvcache, flash_attn_varlen_func
+    except Exception as e:                         # noqa: BLE001 (any import failure)
+        return {"unavailable": f"flash_attn import failed: {e!r}"[:200]}
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+
+        def one(ev):
+            ev[0].record(stream)
+            fn()
+            ev[1].record(stream)
+        return float(np.asarray(timer.time_steps(one, steps))[:, 0].mean())
+
+    res = {"library": "flash_attn " + getattr(__import__("flash_attn"), "__version__", "?"),
+           "note": "black-box comparison on the same buffers; not the oracle, not the product path"}
+    for name in ("gqa7b_decode", "qwen3_0p6b_decode"):
+        w = DecodeWorkload.from_spec(synth.WORKLOADS[name]).upload("cuda")
+        ops.store_kvcache(w.d_new_k, w.d_new_v, w.kc, w.vc, w.d_slots)
+        q4 = w.d_q.unsqueeze(1)
+        lib = flash_attn_with_kvcache(q4, w.kc, w.vc, cache_seqlens=w.d_cl, block_table=w.d_bt,
+                                      causal=True)
+        ours = ops.decode(w.d_q, w.kc, w.vc, w.d_bt, w.d_cl, w.max_context_len, out=w.d_out,
+                          workspace=w.d_ws)
+        torch.cuda.synchronize()
+        diff = float((lib[:, 0].float() - ours.float()).abs().max())
+        t_lib = timed(lambda: flash_attn_with_kvcache(q4, w.kc, w.vc, cache_seqlens=w.d_cl,
+                                                      block_table=w.d_bt, causal=True))
+        t_ours = timed(lambda: ops.decode(w.d_q, w.kc, w.vc, w.d_bt, w.d_cl, w.max_context_len,
+                                          out=w.d_out, workspace=w.d_ws))
+        res[name] = {"flash_attn_ms": round(t_lib, 4), "ours_ms": round(t_ours, 4),
+                     "flash_attn_GBs": round(w.kv_bytes() / (t_lib * 1e-3) / 1e9, 1),
+                     "ours_GBs": round(w.kv_bytes() / (t_ours * 1e-3) / 1e9, 1),
+                     "speedup": round(t_lib / t_ours, 2), "max_abs_diff_outputs": diff}
+        del w
+        torch.cuda.empty_cache()
+    w = PrefixPrefillWorkload(seed=synth.SEED_BASE + 4).upload("cuda")
+    w.store()
+    ours = w.attend().clone()
+    mq, mk = int(w.md.max_seqlen_q), int(w.md.max_seqlen_k)
+    lib = flash_attn_varlen_func(w.d_q, w.kc, w.vc, w.d_cu_q, w.d_cu_k, mq, mk, causal=True,
+                                 block_table=w.d_bt)
+    torch.cuda.synchronize()
+    diff = float((lib.float() - ours.float()).abs().max())
+    t_lib = timed(lambda: flash_attn_varlen_func(w.d_q, w.kc, w.vc, w.d_cu_q, w.d_cu_k, mq, mk,
+                                                 causal=True, block_table=w.d_bt))
+    t_ours = timed(lambda: w.attend())
+    res["prefix_prefill"] = {"flash_attn_ms": round(t_lib, 4), "ours_ms": round(t_ours, 4),
+                             "flash_attn_TFLOPs": round(w.flops() / (t_lib * 1e-3) / 1e12, 1),
+                             "ours_TFLOPs": round(w.flops() / (t_ours * 1e-3) / 1e12, 1),
+                             "speedup": round(t_lib / t_ours, 2), "max_abs_diff_outputs": diff}
+    del w
+    torch.cuda.empty_cache()
+    return res
+
+
 def secondary(torch, args, timer, pk):
     """The other workloads, each at its own roofline (rank 0), at the same --steps / --warmup."""
     from paged_kv_attention_35_b200 import synth
@@ -535,6 +602,11 @@ def secondary(torch, args, timer, pk):
     del w
     torch.cuda.empty_cache()
     nbytes, ms = bench_store_large(torch, steps, warm, timer)
+    try:
+        out["library_comparison"] = library_comparison(torch, steps, warm, timer)
+    except Exception as e:                         # noqa: BLE001 (a library failure is reported)
+        out["library_comparison"] = {"unavailable": repr(e)[:200]}
+        torch.cuda.empty_cache()
     out["store_kvcache_65536"] = {"ms": round(ms, 4), "bytes": nbytes,
                                   "GBs": round(nbytes / (ms * 1e-3) / 1e9, 1),
                                   "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
