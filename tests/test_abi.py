@@ -135,6 +135,30 @@ def test_prefill_validation(ops):
     assert _prefill(ops, tq=0) == 0
 
 
+def _prefill_store(ops, **kw):
+    a = dict(out=256, q=256, qs=3584, key=512, value=512, ks=512, vs=512, slots=64, kc=256, vc=256,
+             cq=64, ck=64, mq=128, mk=256, tq=128, bt=64, mb=4, B=2, hq=28, hkv=4, d=128, bs=256,
+             nb=64, scale=0.088, dtype=0, flag=None)
+    a.update(kw)
+    return ops.lib().pa_prefill_store(a["out"], a["q"], a["qs"], a["key"], a["value"], a["ks"],
+                                      a["vs"], a["slots"], a["kc"], a["vc"], a["cq"], a["ck"], a["mq"],
+                                      a["mk"], a["tq"], a["bt"], a["mb"], a["B"], a["hq"], a["hkv"],
+                                      a["d"], a["bs"], a["nb"], a["scale"], a["dtype"], a["flag"], None)
+
+
+def test_prefill_store_validation(ops):
+    assert _prefill_store(ops, slots=None) == 1               # the store needs its slots
+    assert _prefill_store(ops, key=None) == 1
+    assert _prefill_store(ops, value=520) == 1                # misaligned new rows
+    assert _prefill_store(ops, ks=256) == 1                   # stride < Hkv*D
+    assert _prefill_store(ops, vs=516) == 1                   # stride not a multiple of 8
+    # the prefill checks still apply
+    assert _prefill_store(ops, mq=300, mk=256) == 1
+    assert _prefill_store(ops, hq=6, hkv=4) == 1
+    assert _prefill_store(ops, B=0) == 0                      # nothing to do
+    assert "" == ops.lib().pa_last_error_message().decode()
+
+
 def test_python_binding_refuses_cpu_tensors(ops):
     import torch
     x = torch.zeros(2, 8, 128, dtype=torch.bfloat16)
