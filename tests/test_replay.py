@@ -23,20 +23,38 @@ pytestmark = pytest.mark.gpu
 f64 = oracle.bf16_bits_to_f64
 
 
+_RING_BITS = {}
+
+
+def _ring_bits(rp, which):
+    """The CPU ring of K (or V) rows as one [ring, rows, Hkv, D] uint16 array (cached)."""
+    key = (id(rp), which)
+    if key not in _RING_BITS:
+        ring = rp.k_ring_cpu if which == "k" else rp.v_ring_cpu
+        _RING_BITS.clear()
+        _RING_BITS[key] = np.stack([to_bits(t) for t in ring])
+    return _RING_BITS[key]
+
+
 def _history(rp, snap, block_table, length, layer, which):
-    """[length, Hkv, D] float64 K (or V) rows a sequence's positions hold after a step."""
+    """[length, Hkv, D] float64 K (or V) rows a sequence's positions hold after a step:
+    each position's row is the ring row of the step that last wrote its slot."""
     c = rp.cfg
     slots = oracle.ref_slot_mapping(block_table, range(length), c.block_size)
     writer = snap[slots]
     assert (writer[:, 0] >= 0).all(), "a position was never stored"
-    ring = rp.k_ring_cpu if which == "k" else rp.v_ring_cpu
-    rows = [to_bits(ring[rp.ring_index(int(st), layer)][int(rw)]) for st, rw in writer]
-    return f64(np.stack(rows))
+    steps, inv = np.unique(writer[:, 0], return_inverse=True)
+    ring_idx = np.array([rp.ring_index(int(st), layer) for st in steps])[inv]
+    return f64(_ring_bits(rp, which)[ring_idx, writer[:, 1]])
 
 
-def check_sample(rp, step, layer, max_seqs=None):
+def check_sample(rp, step, layer, max_seqs=None, max_prefill_seqs=None):
+    """Every (or an evenly spread max_seqs / max_prefill_seqs of the) sequence(s) of a
+    captured (step, layer) against the oracle."""
     c = rp.cfg
     smp = rp.samples[(step, layer)]
+    if smp["is_prefill"] and max_prefill_seqs is not None:
+        max_seqs = max_prefill_seqs
     snap = rp.snap[step]
     md = smp["md"]
     q_all = f64(to_bits(rp.q_ring_cpu[rp.ring_index(step, layer)]))
@@ -128,18 +146,22 @@ def test_graph_replay_pools_equal_eager(cuda_device):
 
 
 def test_full_trace_sampled(cuda_device):
-    """512 requests, prompt/output U[100,1024], 256 seqs, block 256, 768 blocks, 28 layers."""
+    """512 requests, prompt/output U[100,1024], 256 seqs, block 256, 768 blocks, 28 layers:
+    nine steps across the trace at layers 0 and 27; 32 evenly spread sequences of a sampled
+    decode step, 8 of a sampled prefill step (about a minute of oracle time)."""
     cfg = ReplayConfig()
     rp = Replay(cfg, record=True)
-    rp.sample_at = {(s, l) for s in (0, 3, 40, 400, 1100) for l in (0, cfg.num_layers - 1)}
+    steps = (0, 3, 40, 400, 800, 1100, 1500, 1900, 2200)
+    rp.sample_at = {(s, l) for s in steps for l in (0, cfg.num_layers - 1)}
     st = rp.run()
     assert st["finished"] == cfg.num_requests
     assert st["preemptions"] > 0
-    checked = 0
+    checked, kinds = 0, set()
     for key in sorted(rp.samples):
-        check_sample(rp, *key, max_seqs=6)
+        check_sample(rp, *key, max_seqs=32, max_prefill_seqs=8)
+        kinds.add(rp.samples[key]["is_prefill"])
         checked += 1
-    assert checked >= 6
+    assert checked >= 16 and kinds == {True, False}
 
 
 def test_full_trace_graphs_sampled(cuda_device):
