@@ -263,7 +263,9 @@ PA_API pa_status pa_prefill_varlen(void* out, const void* q, int64_t q_token_str
  * block_size + p % block_size for p = k_len-q_len+j (the Block Manager's
  * mapping, "From Sequences to Blocks", lnwmold.com item; the step's new K/V
  * are written before attention reads them, "Preparation before computation",
- * same item).  Attention reads the new keys and values straight from key /
+ * same item) and no new token's slot lies in a block that another sequence of
+ * the batch reads as its cached prefix (the block manager only shares full,
+ * already-written blocks).  Attention reads the new keys and values straight from key /
  * value and the cached prefix from the pool, so nothing waits for the store;
  * each new (token, KV head) row is written to the pool once, by the CTA that
  * computes that token's queries, during the same launch.  A TMA box of pool
