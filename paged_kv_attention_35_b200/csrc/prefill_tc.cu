@@ -663,15 +663,17 @@ __global__ void __launch_bounds__(kTcBoundThreads, 1)
   } else if (warp == 9 || warp == 10) {
     // ------------------------------------------------------------ MMA issuers
     // Warp 9 issues tile A's MMAs, warp 10 tile B's (lane 0; the warp takes
-    // the unit descriptors).  Per tile: S_t(j+1) before P_t(j) V_j, so the
-    // tile's next S is ready when its softmax finishes.  The S columns are
-    // used in one fixed order, A0 B0 A1 B1 ... (A alone once B has no more KV
-    // tiles), and every S waits until the previous S in that order has been
-    // read into registers; each P V waits only for its own tile's P.  (The
-    // protocol was checked by a model of all roles and of the asynchronous
-    // copies and MMAs under random schedules: no deadlock, no wait whose
-    // parity could alias another phase, and no unordered conflicting access
-    // other than the two tiles' identical zero writes to the last V tile.)
+    // the unit descriptors).  Per tile, S_t(j+1) and P_t(j) V_j are issued in
+    // whichever order their inputs become ready, so the tile's next S is
+    // usually computed while its softmax runs and a P V never waits behind the
+    // S columns.  The S columns are used in one fixed order, A0 B0 A1 B1 ...
+    // (A alone once B has no more KV tiles), and every S waits until the
+    // previous S in that order has been read into registers; each P V waits
+    // only for its own tile's P.  (The protocol was checked by a model of all
+    // roles and of the asynchronous copies and MMAs under random schedules: no
+    // deadlock, no wait whose parity could alias another phase, and no
+    // unordered conflicting access other than the two tiles' identical zero
+    // writes to the last V tile.)
     const int t = warp - 9;
     constexpr uint32_t idS = tc::idesc_bf16(kTcRows, kTcKeys, false, false);
     constexpr uint32_t idO = tc::idesc_bf16(kTcRows, D, false, true);
