@@ -212,3 +212,25 @@ def test_fused_block_table_past_staged_entries(cuda_device):
     got = _fused(c, key, value, slots, q, cu_q, cu_k, bt)
     assert got[3] == 0
     _check_same(got, ref, "block 16, 5000 tokens")
+
+
+def test_fused_random_configs(cuda_device):
+    """Twelve seeded random batches: block size 16..1024, head shapes with groups of 1 to 16,
+    D 64 or 128, 1-6 sequences with cached lengths 0..700 (aligned to the box or not) and
+    1..400 new tokens; output and pools bit-identical to store-then-prefill, no flags."""
+    import random
+    rnd = random.Random(2024)
+    shapes = [(8, 8, 64), (16, 8, 128), (28, 4, 128), (32, 2, 64), (16, 1, 128), (12, 3, 128)]
+    for case in range(12):
+        hq, hkv, d = rnd.choice(shapes)
+        bs = rnd.choice([16, 32, 64, 128, 256, 1024])
+        nseq = rnd.randint(1, 6)
+        cached = [rnd.choice([0, 0, rnd.randint(1, 700), 128 * rnd.randint(1, 5)]) for _ in range(nseq)]
+        new = [rnd.randint(1, 400) for _ in range(nseq)]
+        c = PrefillCase(cached, new, hq=hq, hkv=hkv, d=d, bs=bs, seed=300 + case)
+        key, value, slots = _new_rows(c)
+        q, cu_q, cu_k, bt = _inputs(c)
+        ref = _two_launch(c, key, value, slots, q, cu_q, cu_k, bt)
+        got = _fused(c, key, value, slots, q, cu_q, cu_k, bt)
+        assert got[3] == 0, (case, got[3])
+        _check_same(got, ref, f"random case {case}: {hq}/{hkv} d{d} bs{bs} {cached} {new}")
