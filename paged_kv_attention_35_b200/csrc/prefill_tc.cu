@@ -160,12 +160,15 @@ struct TcWalk {
   int64_t base;  // list position of the window's first unit
   bool have;     // the lane values below belong to (b, s0)
   int cnt, lo, incl, total;   // this lane's sequence in the window: units, first pair, prefix
+  int q_s0;      // the window whose lengths q holds (-1: none): with at most 32 sequences
+                 // the lengths are read once, not once per bucket
   TcSeq q;
   __device__ __forceinline__ void init(const PrefillTcParams& p) {
     b = p.buckets;
     s0 = 0;
     base = 0;
     have = false;
+    q_s0 = -1;
   }
   // Fills u with the unit at list position pos; false past the end.  With
   // `report`, invalid sequence lengths raise PA_FLAG_LEN_OOB (once per CTA).
@@ -176,15 +179,15 @@ struct TcWalk {
         const int s = s0 + lane;
         cnt = 0;
         lo = 0;
-        if (s < p.num_seqs) {
-          q = tc_seq(p, s);
-          if (!q.ok && report && b == p.buckets) raise_flag(p.err_flag, PA_FLAG_LEN_OOB);
-          if (q.P > 0) {
-            lo = tc_first_pair(q, b, p.qpt);
-            cnt = (tc_first_pair(q, b - 1, p.qpt) - lo) * p.hkv;
-          }
-        } else {
-          q = TcSeq{};
+        if (q_s0 != s0) {
+          q = s < p.num_seqs ? tc_seq(p, s) : TcSeq{};
+          if (s < p.num_seqs && !q.ok && report && b == p.buckets)
+            raise_flag(p.err_flag, PA_FLAG_LEN_OOB);
+          q_s0 = s0;
+        }
+        if (s < p.num_seqs && q.P > 0) {
+          lo = tc_first_pair(q, b, p.qpt);
+          cnt = (tc_first_pair(q, b - 1, p.qpt) - lo) * p.hkv;
         }
         incl = cnt;
 #pragma unroll
@@ -343,6 +346,11 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 
 // 2^x for two values on the FMA pipe.  x is clamped to >= -125 (2^-125 is
 // below anything that survives the bf16 rounding of P next to a 1; below the
@@ -396,13 +404,23 @@ __device__ __forceinline__ void st_stream16(uint4* a, uint4 v) {
                : "memory");
 }
 
+// One 32-byte global store (a full sector per lane): the epilogue's rows sit
+// 256 bytes apart across a warp, so each store instruction touches 32 lines
+// whatever its width, and 32-byte stores halve the instructions and the L1
+// wavefronts of 16-byte ones.  `a` must be 32-byte aligned.
+__device__ __forceinline__ void st_global32(void* a, uint4 lo, uint4 hi) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(a), "r"(lo.x),
+               "r"(lo.y), "r"(lo.z), "r"(lo.w), "r"(hi.x), "r"(hi.y), "r"(hi.z), "r"(hi.w)
+               : "memory");
+}
+
 // Fused store: copies the new K/V rows of a sequence's new tokens [r0, r1)
 // (token r is key position cached + r) for KV head kvh to their pool slots.
-// Per group of 32 tokens, lane j reads token j's slot (and, with `check`, its
-// block-table slot: a slot that differs raises PA_FLAG_SLOT_MISMATCH, one past
-// the pool PA_FLAG_SLOT_OOB) in one coalesced load; then the rows are copied
-// in 16-byte chunks spread over the warp, kBatch loads in flight per lane.
-// Negative and out-of-pool slots write nothing.
+// Per round of kRound tokens the warp reads the rows in 16-byte chunks spread
+// over its lanes (kBatch loads in flight per lane) while lane j reads token
+// j's slot (and, with `check`, its block-table slot: a slot that differs
+// raises PA_FLAG_SLOT_MISMATCH, one past the pool PA_FLAG_SLOT_OOB), then
+// writes the rows.  Negative and out-of-pool slots write nothing.
 template <int D>
 __device__ __forceinline__ void tc_store_rows(const PrefillTcParams& p, int q_start, int cached,
                                               const int32_t* bt, int kvh, int r0, int r1, int lane,
@@ -410,14 +428,24 @@ __device__ __forceinline__ void tc_store_rows(const PrefillTcParams& p, int q_st
   constexpr int C = D / 8;             // chunks of one K or V row
   constexpr int kPer = 2 * C;          // chunks of a token: K, then V
   constexpr int kTok = 32 / kPer;      // tokens one warp-wide access covers
-  constexpr int kBatch = 8;
+  constexpr int kBatch = 16;           // accesses in flight per lane
+  constexpr int kRound = kBatch * kTok;   // tokens per round (at most 32: one slot per lane)
+  static_assert(kRound <= 32, "one slot per lane");
   const int c = lane % kPer, ch = c % C;
   const bool isv = c >= C;
   const uint4* src = (isv ? p.new_v : p.new_k) + kvh * C + ch;
   const int64_t sstride = isv ? p.new_v_stride16 : p.new_k_stride16;
   uint4* pool = (isv ? p.vc : p.kc) + kvh * C + ch;
-  for (int g = r0; g < r1; g += 32) {
-    const int n = min(32, r1 - g);
+  for (int g = r0; g < r1; g += kRound) {
+    const int n = min(kRound, r1 - g);
+    // the round's rows are read before, and independently of, their slots, so
+    // the slot loads and the row loads are in flight together (one round trip)
+    uint4 v[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int t = u * kTok + lane / kPer;
+      if (t < n) v[u] = ld_stream16(src + (int64_t)(q_start + g + t) * sstride);
+    }
     int slot = -1;
     if (lane < n) {
       slot = __ldg(p.slots + q_start + g + lane);
@@ -431,19 +459,11 @@ __device__ __forceinline__ void tc_store_rows(const PrefillTcParams& p, int q_st
           raise_flag(p.err_flag, PA_FLAG_SLOT_MISMATCH);
       }
     }
-    for (int t0 = 0; t0 < n; t0 += kBatch * kTok) {
-      uint4 v[kBatch];
-      int sl[kBatch];
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int t = t0 + u * kTok + lane / kPer;       // token within the group (< 32 + kBatch)
-        sl[u] = __shfl_sync(0xffffffffu, slot, t & 31);
-        if (t >= n) sl[u] = -1;
-        if (sl[u] >= 0) v[u] = ld_stream16(src + (int64_t)(q_start + g + t) * sstride);
-      }
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u)
-        if (sl[u] >= 0 && sl[u] < p.num_slots) st_stream16(pool + (int64_t)sl[u] * p.hkv * C, v[u]);
+    for (int u = 0; u < kBatch; ++u) {
+      const int t = u * kTok + lane / kPer;
+      const int sl = __shfl_sync(0xffffffffu, slot, t);
+      if (t < n && sl >= 0 && sl < p.num_slots) st_stream16(pool + (int64_t)sl * p.hkv * C, v[u]);
     }
   }
 }
@@ -988,15 +1008,32 @@ __global__ void __launch_bounds__(kTcBoundThreads, 1)
         for (int c = 0; c < D / 32; ++c) tc::ld32(tO + c * 32, ov + c * 32);
       }
       tc::wait_ld();
-      if (store) {
+      // O / l, two columns per packed multiply
+      const uint64_t inv2 = f32x2(inv, inv);
 #pragma unroll
-        for (int k = 0; k < D / 8; ++k) {
-          uint4 v;
-          v.x = pack_bf16(__uint_as_float(ov[8 * k + 0]) * inv, __uint_as_float(ov[8 * k + 1]) * inv);
-          v.y = pack_bf16(__uint_as_float(ov[8 * k + 2]) * inv, __uint_as_float(ov[8 * k + 3]) * inv);
-          v.z = pack_bf16(__uint_as_float(ov[8 * k + 4]) * inv, __uint_as_float(ov[8 * k + 5]) * inv);
-          v.w = pack_bf16(__uint_as_float(ov[8 * k + 6]) * inv, __uint_as_float(ov[8 * k + 7]) * inv);
-          *reinterpret_cast<uint4*>(orow + k * 8) = v;
+      for (int m = 0; m < D / 2; ++m) {
+        float a, b;
+        f32x2_split(fmul2(f32x2(__uint_as_float(ov[2 * m]), __uint_as_float(ov[2 * m + 1])), inv2), a, b);
+        ov[2 * m] = __float_as_uint(a);
+        ov[2 * m + 1] = __float_as_uint(b);
+      }
+      // 8 output columns of this row as bf16
+      auto pack8 = [&](int k) {
+        uint4 v;
+        v.x = pack_bf16(__uint_as_float(ov[8 * k + 0]), __uint_as_float(ov[8 * k + 1]));
+        v.y = pack_bf16(__uint_as_float(ov[8 * k + 2]), __uint_as_float(ov[8 * k + 3]));
+        v.z = pack_bf16(__uint_as_float(ov[8 * k + 4]), __uint_as_float(ov[8 * k + 5]));
+        v.w = pack_bf16(__uint_as_float(ov[8 * k + 6]), __uint_as_float(ov[8 * k + 7]));
+        return v;
+      };
+      if (store) {
+        // rows are D * 2 bytes apart: 32-byte stores when the base allows
+        if ((reinterpret_cast<uintptr_t>(p.out) & 31u) == 0) {
+#pragma unroll
+          for (int k = 0; k < D / 8; k += 2) st_global32(orow + k * 8, pack8(k), pack8(k + 1));
+        } else {
+#pragma unroll
+          for (int k = 0; k < D / 8; ++k) *reinterpret_cast<uint4*>(orow + k * 8) = pack8(k);
         }
       }
       // the next unit's first P V overwrites O_t: every lane's reads are done

@@ -138,3 +138,22 @@ def test_prefill_block_table_past_staged_entries(cuda_device):
     block-table entries the producer stages in shared memory (the rest are read directly)."""
     c = PrefillCase([1000, 3], [4000, 4997], hq=8, hkv=2, d=64, bs=16, seed=41)
     compare(c.run_gpu(), c.oracle_prefill(), "prefill past staged block-table entries")
+
+
+@pytest.mark.parametrize("hq,hkv,d", [(28, 4, 128), (8, 1, 64)])
+def test_prefill_output_only_16_byte_aligned(cuda_device, hq, hkv, d):
+    """An output buffer that is 16- but not 32-byte aligned takes the 16-byte store path of
+    the epilogue (32-byte stores otherwise): the same bits either way."""
+    from paged_kv_attention_35_b200 import ops
+    c = PrefillCase([0, 17, 300], [129, 47, 200], hq=hq, hkv=hkv, d=d, bs=64, seed=5 + d)
+    ref = c.run_gpu()
+    assert ref.data_ptr() % 32 == 0
+    buf = torch.zeros(ref.numel() + 8, dtype=torch.bfloat16, device=ref.device)
+    out = buf[8:].view(ref.shape)
+    assert out.data_ptr() % 32 == 16
+    ops.prefill_varlen(c.q.to(ref.device), c.kc, c.vc, torch.from_numpy(c.cu_q).to(ref.device),
+                       torch.from_numpy(c.cu_k).to(ref.device), max(c.new), max(c.k_lens),
+                       torch.from_numpy(c.block_tables).to(ref.device), out=out)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    assert torch.equal(buf[:8].view(torch.int16), torch.zeros(8, dtype=torch.int16, device=ref.device))
