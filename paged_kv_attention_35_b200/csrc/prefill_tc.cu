@@ -39,16 +39,17 @@
 //   warps 9, 10   MMA issuers of tiles A and B (one thread each): S_t(j) =
 //            Q_t K_j^T into the TMEM S columns (M=128, N=128, K=16 steps);
 //            O_t += P_t(j) V_j with P read from TMEM (TS form, B = V MN-major);
-//            per tile S_t(j+1) goes before P_t(j) V_j, so the tensor core works
-//            on one tile while the other tile's softmax runs, and neither
-//            tile's P V waits for the other's softmax.
+//            per tile S_t(j+1) and P_t(j) V_j are issued in whichever order
+//            their inputs become ready (the S columns' turn; P_t), so the
+//            tensor core works on one tile while the other tile's softmax runs
+//            and no P V waits behind the S columns.
 //   warps 0-3 / 4-7   softmax of tile A / B, one thread per M row (TMEM lane):
 //            causal mask on the tiles that reach past a row's last key; online
 //            softmax in the log2 domain with a lazy rescale (the reference max
 //            moves only when it grows by more than 8, i.e. 256x); exponentials
 //            on the MUFU unit (a polynomial on the FMA pipe, Exp2Poly, can take
 //            a share of them: kEmuPairs); P as bf16 pairs in the tile's TMEM
-//            P columns; epilogue O / l -> bf16 -> global.
+//            P columns; epilogue O / l -> bf16 -> global in 32-byte stores.
 //            The warps of a tile that reads the unit's last V tile zero its rows
 //            past the unit's last key (up to the next multiple of 16: P V skips
 //            the 16-key steps beyond) before handing over P (stale pool rows may
