@@ -85,7 +85,7 @@ def cta_units(cached, new, group, cta, grid):
         mine.append(lst[pos])
 
 
-def run(units, rnd, mistake=None, fused=False):
+def run(units, rnd, mistake=None):
     """Runs one CTA's roles over `units`; returns None, or the roles stuck in a deadlock.
 
     Besides the parity checks, the shared S columns are tracked as data: writing an S
@@ -94,11 +94,9 @@ def run(units, rnd, mistake=None, fused=False):
     that show the model can fail: "no_read_counter" issues an S without waiting for the
     previous S's readers, "single_release" has tile A free the ring slots of the K/V
     tiles tile B skips once instead of twice, "early_p" writes P without waiting for the
-    previous P V, and "store_not_counted" leaves the empty barriers at two arrivals although
-    the store warp also arrives on them."""
+    previous P V."""
     bars, reads = {}, {0: 0, 1: 0}
     s_cols = {"owner": None, "reads": 4}
-    ring = [None] * KRING                      # the fill index each ring slot holds
 
     def bar(name, count=1):
         return bars.setdefault(name, Bar(name, count))
@@ -109,10 +107,10 @@ def run(units, rnd, mistake=None, fused=False):
         bar(f"p_full{t}", 4)
     for s in range(KRING):
         bar(f"kv_full{s}")
-        bar(f"kv_empty{s}", 3 if fused and mistake != "store_not_counted" else 2)
+        bar(f"kv_empty{s}", 2)
     for s in range(USLOTS):
         bar(f"unit_full{s}")
-        bar(f"unit_empty{s}", READERS + (1 if fused else 0))
+        bar(f"unit_empty{s}", READERS)
     desc = [None] * USLOTS
 
     def wait(name, k):
@@ -142,7 +140,6 @@ def run(units, rnd, mistake=None, fused=False):
                 slot = kv_i % KRING
                 if kv_i >= KRING:
                     yield wait(f"kv_empty{slot}", kv_i // KRING - 1)
-                yield ("fill", slot, kv_i)
                 yield arrive(f"kv_full{slot}")
                 kv_i += 1
 
@@ -242,24 +239,7 @@ def run(units, rnd, mistake=None, fused=False):
                 yield wait(f"pv_done{t}", pvc)
                 pvc += 1
 
-    def store():
-        # the fused store warp: takes every unit and, for each of its K/V ring
-        # entries in order, waits for the tile, copies the unit's own new rows
-        # out of it and frees the slot (a third arrival on its empty barrier)
-        kv_i = 0
-        for k in itertools.count():
-            n, _, _ = yield from take(k)
-            if n == 0:
-                return
-            for idx in range(kv_i, kv_i + 2 * n):
-                yield wait(f"kv_full{idx % KRING}", idx // KRING)
-                yield ("copy", idx % KRING, idx)
-                yield arrive(f"kv_empty{idx % KRING}")
-            kv_i += 2 * n
-
     roles = {"producer": producer(), "issuerA": issuer(0), "issuerB": issuer(1)}
-    if fused:
-        roles["store"] = store()
     for t in (0, 1):
         for w in range(4):
             roles[f"softmax{'AB'[t]}{w}"] = softmax(t)
@@ -288,12 +268,7 @@ def run(units, rnd, mistake=None, fused=False):
                 if op[0] == "spin":
                     pending[r] = None
                     break
-                if op[0] == "fill":
-                    ring[op[1]] = op[2]
-                elif op[0] == "copy":
-                    assert ring[op[1]] == op[2], \
-                        f"store reads fill {op[2]} of slot {op[1]}, which holds {ring[op[1]]}"
-                elif op[0] == "write_s":
+                if op[0] == "write_s":
                     assert s_cols["reads"] == 4, \
                         f"S {op[1:]} written over S {s_cols['owner']} before all its readers"
                     s_cols["owner"], s_cols["reads"] = op[1:], 0
@@ -332,30 +307,11 @@ def test_random_unit_lists():
         assert run(units, rnd) is None, units
 
 
-def test_fused_store_warp_on_the_ring():
-    """The store warp as a third consumer of every K/V ring slot and an eleventh unit reader:
-    no deadlock, and every copy reads the fill it waited for."""
-    rnd = random.Random(17)
-    cached = [0, 0, 0, 17, 256, 300, 0, 5, 1024]
-    new = [1, 63, 129, 47, 1, 200, 256, 64, 65]
-    for seed in range(4):
-        for group in (1, 7):
-            for grid in (1, 148):
-                assert run(cta_units(cached, new, group, 0, grid), random.Random(seed), fused=True) is None
-    for _ in range(200):
-        units = []
-        for _ in range(rnd.randint(1, 8)):
-            na = rnd.randint(1, 12)
-            nb = rnd.choice([0, na, max(0, na - 1), rnd.randint(0, na)])
-            units.append((na, nb, (na - 1) * 128 + rnd.randint(1, 128)))
-        assert run(units, rnd, fused=True) is None, units
-
-
-def _fails(units, mistake, seeds=20, fused=False):
+def _fails(units, mistake, seeds=20):
     """True when some schedule of `units` with `mistake` planted trips a check."""
     for seed in range(seeds):
         try:
-            if run(units, random.Random(seed), mistake, fused) is not None:
+            if run(units, random.Random(seed), mistake) is not None:
                 return True
         except AssertionError:
             return True
@@ -367,5 +323,3 @@ def test_the_model_catches_planted_mistakes():
     for mistake in ("no_read_counter", "single_release", "early_p"):
         assert _fails(units, mistake), mistake
     assert not _fails(units, None)
-    assert _fails(units, "store_not_counted", fused=True)
-    assert not _fails(units, None, fused=True)
