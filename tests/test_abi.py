@@ -194,3 +194,34 @@ def test_decode_store_validation(ops):
 def test_selftest_validation(ops):
     assert ops.lib().pa_selftest_wait_timeout(None, 0, None, None) == 1
     assert ops.lib().pa_selftest_wait_timeout(None, 3_000_000, None, None) == 1
+
+
+def test_header_is_plain_c_and_links(ops, tmp_path):
+    """The boundary needs no Python or C++: a strict C99 program includes the header, links
+    the library, and gets a workspace size and a host-side argument error back from it."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "consumer.c"
+    src.write_text(r'''
+#include "pagedattn.h"
+#include <stdio.h>
+int main(void) {
+  size_t need = pa_decode_workspace_size(256, 28, 4, 128, 4096, 0);
+  pa_status s = pa_store_kvcache(0, 0, 0, 0, 0, 0, 0, 1, 4, 128, 1024, PA_BF16, 0, 0);
+  printf("%zu %d %s\n", need, (int)s, pa_status_string(s));
+  return s == PA_OK;
+}
+''')
+    exe = tmp_path / "consumer"
+    libdir = os.path.dirname(LIB)
+    subprocess.run([cc, "-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                    "-L", libdir, "-lpagedattn", "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    need, code, name = out.stdout.split()
+    assert int(need) > 0
+    assert ops.STATUS[int(code)] == "PA_ERR_INVALID_ARG" == name
