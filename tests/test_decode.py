@@ -51,6 +51,13 @@ def test_large_group_over_16(cuda_device):
     compare(c.run_gpu(), c.oracle_decode(), "group 20")
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_largest_group(cuda_device, d):
+    """128 query heads on one KV head: eight query tiles per KV head."""
+    c = DecodeCase([1, 300, 1000], hq=128, hkv=1, d=d, bs=16, seed=13 + d)
+    compare(c.run_gpu(), c.oracle_decode(), f"group 128 d{d}")
+
+
 def test_layout_and_permutation_invariance(cuda_device):
     """Same logical K/V and q under block sizes 16 / 256 / one block per sequence
     and under two shuffles of the pool: each within tolerance of the oracle, and

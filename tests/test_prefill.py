@@ -122,6 +122,14 @@ def test_prefill_group_packing(cuda_device, hq, hkv, d):
     compare(out, c.oracle_prefill(), f"prefill {hq}/{hkv} d{d}")
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_largest_group(cuda_device, d):
+    """128 query heads on one KV head, the most a tile packs: one query per tile, so
+    every pair of queries is a unit."""
+    c = PrefillCase([0, 5, 130], [3, 40, 17], hq=128, hkv=1, d=d, bs=16, seed=61 + d)
+    compare(c.run_gpu(), c.oracle_prefill(), f"prefill group 128 d{d}")
+
+
 def test_prefill_many_sequences(cuda_device):
     """More work units than SMs: each persistent CTA walks many units."""
     rng = np.random.default_rng(99)
